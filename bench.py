@@ -1,0 +1,393 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A4 group-quantized GEMM hot path on B200.
+
+One step = the whole hot path over one batch: online per-token activation quantization
+(apex_quantize_act_int4) followed by the W4A4 GEMM (apex_w4a4_gemm); the weights are
+packed once, offline.  Metric: effective TOPS = 2*M*N*K / step time, reported with the
+roofline fraction of the dominant kernel (the GEMM).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl apex|reference]
+
+Inputs larger than L2: every step uses the next of several copies of the packed weights
+and activations, so each step reads its operands from HBM.  Under torchrun each rank runs
+an independent replica (the path has no exchange step), time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from group_quantized_w4a4_b200 import roofline, synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "decode_m16_n8192_k8192"
+SECOND_WORKLOAD = "prefill_m4096_n8192_k8192"
+INT8_PER_BF16 = 2.0   # nominal dense int8 : bf16 tensor throughput ratio on B200 (4.5 : 2.25)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_init(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ the apex arm
+
+class Problem:
+    """Device-resident operands for one workload, in C copies (inputs larger than L2)."""
+
+    def __init__(self, apex, torch, g: synth.Gemm, copies: int):
+        self.g = g
+        a, w = synth.make(g)
+        self.a_host = a
+        dev = torch.device("cuda")
+        self.x = []
+        self.wp, self.sw, self.ap, self.sa = [], [], [], []
+        a_d = torch.from_numpy(a).to(dev)
+        w_d = torch.from_numpy(w).to(dev)
+        wp0, sw0 = apex.pack_weights(w_d, g.gw)
+        del w_d
+        for c in range(copies):
+            self.x.append(a_d if c == 0 else a_d.clone())
+            self.wp.append(wp0 if c == 0 else wp0.clone())
+            self.sw.append(sw0 if c == 0 else sw0.clone())
+            self.ap.append(torch.empty((g.M, g.K // 2), dtype=torch.uint8, device=dev))
+            self.sa.append(torch.empty((g.M, g.K // 128), dtype=torch.float16, device=dev))
+        self.y = torch.empty((g.M, g.N), dtype=torch.float16, device=dev)
+        self.ws = apex.workspace(g.M, g.N, g.K, 128, g.gw)
+        self.copies = copies
+
+
+def copies_for(g: synth.Gemm, l2_bytes: int) -> int:
+    per = g.gemm_bytes() + g.quant_bytes()
+    c = 2
+    while c * per < 2 * l2_bytes and c < 64:
+        c += 1
+    return c
+
+
+def apex_step(apex, p: Problem, i: int, stream, ev=None):
+    g = p.g
+    c = i % p.copies
+    apex.apex_quantize_act_int4(p.x[c], g.M, g.K, 128, p.ap[c], p.sa[c], stream)
+    if ev is not None:
+        ev[0].record(stream)
+    apex.apex_w4a4_gemm(g.M, g.N, g.K, 128, g.gw, p.ap[c], p.sa[c], p.wp[c], p.sw[c], p.y,
+                        p.ws, None, stream)
+    if ev is not None:
+        ev[1].record(stream)
+
+
+def time_workload(apex, torch, g, steps, warmup, world, l2_bytes, clocks=None):
+    p = Problem(apex, torch, g, copies_for(g, l2_bytes))
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        apex_step(apex, p, i, stream)
+    torch.cuda.synchronize()
+    if apex.apex_get_device_status(stream) != 0:
+        raise RuntimeError("device status not clean after warm-up")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+    start.record(stream)
+    for i in range(steps):
+        apex_step(apex, p, warmup + i, stream, evs[i])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    if apex.apex_get_device_status(stream) != 0:
+        raise RuntimeError("device status not clean after the timed steps")
+    total_ms = start.elapsed_time(stop)
+    gemm_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    return p, total_ms, gemm_ms, clk
+
+
+def e2e_workload(apex, torch, g, steps, warmup, p: Problem):
+    """Same step through the public API with host buffers: pinned fp16 activations copied
+    in, quantize + GEMM, fp16 output copied back, all inside the timed region."""
+    stream = torch.cuda.current_stream()
+    x_host = torch.from_numpy(p.a_host).pin_memory()
+    y_host = torch.empty((g.M, g.N), dtype=torch.float16).pin_memory()
+
+    def step(i):
+        c = i % p.copies
+        p.x[c].copy_(x_host, non_blocking=True)
+        apex_step(apex, p, i, stream)
+        y_host.copy_(p.y, non_blocking=True)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        step(warmup + i)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(stop) / steps
+    return ms, x_host.numel() * 2, y_host.numel() * 2
+
+
+def roofline_obj(g, gemm_ms_avg, peaks, peaks_kind, traffic=None):
+    hbm = float(peaks["hbm_gbs"]) * 1e9
+    i8 = float(peaks.get("bf16_tflops", 1590.0)) * 1e12 * INT8_PER_BF16
+    t_bound, bound = roofline.bound_time_s(g.ops, g.gemm_bytes(), i8, hbm)
+    t = gemm_ms_avg * 1e-3
+    if bound == "hbm":
+        achieved = g.gemm_bytes() / t / 1e9
+        peak = float(peaks["hbm_gbs"])
+        unit = "GB/s"
+        note = f"hbm_gbs of {peaks_kind}"
+    else:
+        achieved = g.ops / t / 1e12
+        peak = i8 / 1e12
+        unit = "TOPS"
+        note = f"int8 = {INT8_PER_BF16:g} x bf16_tflops of {peaks_kind} (nominal int8:bf16 ratio)"
+    return {"bound": "hbm" if bound == "hbm" else "tensor", "achieved": round(achieved, 2),
+            "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
+            "traffic": traffic, "peak_source": note,
+            "algorithmic_bytes": g.gemm_bytes(), "ops": g.ops,
+            "kernel_ms": round(gemm_ms_avg, 5)}
+
+
+def cpu_baseline(g: synth.Gemm, budget_s: float = 20.0):
+    """The oracle, as it stands, on this host's cores: quantize the activations and run the
+    fp64 GEMM over a bounded sample of output rows; effective TOPS scaled to the rows."""
+    import oracle
+    a, w = synth.make(g)
+    wp, sw = oracle.quantize_pack(w, g.gw)
+    rows = np.arange(min(g.M, 4), dtype=np.int64)
+    t0 = time.perf_counter()
+    ap, sa = oracle.quantize_pack(a[rows], 128)
+    oracle.gemm(ap, sa, wp, sw, rows.size, g.N, g.K, 128, g.gw)
+    dt = time.perf_counter() - t0
+    n = rows.size
+    # grow the sample while it stays well inside the budget
+    while n < g.M and dt * 2 < budget_s / 4:
+        n = min(g.M, n * 2)
+        rows = np.arange(n, dtype=np.int64)
+        t0 = time.perf_counter()
+        ap, sa = oracle.quantize_pack(a[rows], 128)
+        oracle.gemm(ap, sa, wp, sw, n, g.N, g.K, 128, g.gw)
+        dt = time.perf_counter() - t0
+    tops = 2.0 * n * g.N * g.K / dt / 1e12
+    return {"value": round(tops, 6), "unit": "TOPS", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{n} of {g.M} token rows x all {g.N} outputs of {g.name} "
+                      f"(quantize + int64 partials + fp64 scaling), {dt:.2f} s"}
+
+
+def run_apex(args, rank, world, local):
+    import torch
+    import group_quantized_w4a4_b200 as apex
+    apex.load_library()
+    torch.cuda.set_device(local)
+    props = torch.cuda.get_device_properties(local)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 1024 * 1024))
+    peaks, peaks_kind = load_peaks()
+    g = synth.workloads()[args.workload]
+    clocks = ClockSampler(local) if rank == 0 else None
+    p, total_ms, gemm_ms, clk = time_workload(apex, torch, g, args.steps, args.warmup, world,
+                                              l2, clocks)
+    ms_step = max_over_ranks(total_ms / args.steps, world)
+    gemm_avg = statistics.mean(gemm_ms)
+    value = world * g.ops / (ms_step * 1e-3) / 1e12
+    e2e_ms, hb, db = e2e_workload(apex, torch, g, max(3, args.steps), args.warmup, p)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    del p
+    torch.cuda.empty_cache()
+    extra = {}
+    if not args.no_second and args.workload != SECOND_WORKLOAD:
+        g2 = synth.workloads()[SECOND_WORKLOAD]
+        p2, tot2, gm2, _ = time_workload(apex, torch, g2, max(3, args.steps // 4),
+                                         args.warmup, world, l2)
+        ms2 = max_over_ranks(tot2 / max(3, args.steps // 4), world)
+        extra[SECOND_WORKLOAD] = {
+            "value": round(world * g2.ops / (ms2 * 1e-3) / 1e12, 2), "unit": "TOPS",
+            "ms_per_step": round(ms2, 4),
+            "roofline": roofline_obj(g2, statistics.mean(gm2), peaks, peaks_kind)}
+        del p2
+    if rank != 0:
+        return None
+    line = {
+        "metric": "W4A4-g128 GEMM effective TOPS (quantize + GEMM step) and % of roofline",
+        "value": round(value, 2), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8 MMA (int4 operands), fp32 epilogue",
+        "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights, fp16)",
+        "config": {"workload": g.name, "M": g.M, "N": g.N, "K": g.K, "group_a": 128,
+                   "group_w": g.gw, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2: {p_copies(g, l2)} rotating copies"},
+        "roofline": roofline_obj(g, gemm_avg, peaks, peaks_kind),
+        "e2e": {"value": round(world * g.ops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
+                "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db,
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+        "impl": "apex",
+    }
+    if extra:
+        line["also"] = extra
+    if world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(g)
+    return line
+
+
+def p_copies(g, l2):
+    return copies_for(g, l2)
+
+
+def run_reference(args, rank, world):
+    """The oracle, as it stands, on the host cores, for the same workload and metric."""
+    if rank != 0:
+        return None
+    g = synth.workloads()[args.workload]
+    vals = []
+    for _ in range(args.warmup):
+        cpu_baseline(g, budget_s=4.0)
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(g, budget_s=8.0))
+    v = statistics.median([x["value"] for x in vals])
+    cb = dict(vals[-1])
+    cb["value"] = v
+    return {"metric": "W4A4-g128 GEMM effective TOPS (quantize + GEMM step) and % of roofline",
+            "value": v, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int64 partials, fp64 scaling", "data": "synthetic",
+            "config": {"workload": g.name, "M": g.M, "N": g.N, "K": g.K, "group_a": 128,
+                       "group_w": g.gw},
+            "impl": "reference", "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.workloads()))
+    ap.add_argument("--impl", default="apex", choices=["apex", "reference"])
+    ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
+    ap.add_argument("--no-second", action="store_true", help="skip the M=4096 companion line")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_init(args.gpus)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_apex(args, rank, world, local)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,314 @@
+// apex_w4a4.cu -- host side of the C ABI declared in include/apex_w4a4.h: argument
+// validation, TMA descriptor encoding, tile/split selection and kernel launches.
+// All device code lives in the headers included below (one translation unit, so the
+// library-wide device status word needs no separate device linking).
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "apex_w4a4.h"
+#include "gemm.cuh"
+#include "ptx.cuh"
+#include "quantize.cuh"
+
+namespace {
+
+using apex::GemmArgs;
+using apex::GemmCfg;
+
+uint64_t g_wait_limit_ns = 2000000000ull;
+thread_local int t_withhold = -1;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+apex_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return APEX_OK;
+  return APEX_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ device properties
+
+struct DevInfo {
+  int sms = 0;
+};
+
+DevInfo dev_info() {
+  static std::mutex mu;
+  static DevInfo cache[64];
+  static bool have[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DevInfo{148};
+  std::lock_guard<std::mutex> lk(mu);
+  if (!have[dev]) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+    cache[dev].sms = sms;
+    have[dev] = true;
+  }
+  return cache[dev];
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a packed int4 matrix [rows][K/2] bytes; box = 64 bytes (one 128-wide
+// K-group) x box_rows rows, 64-byte swizzle, out-of-range rows read as zeros.
+bool make_packed_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ GEMM planning
+
+struct Plan {
+  int bt = 128;
+  int splits = 1;
+  int tiles_n = 0, tiles_m = 0;
+};
+
+int pick_bt(int64_t M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  return 128;
+}
+
+int ctas_per_sm(int bt) { return bt <= 32 ? 2 : 1; }
+
+Plan make_plan(int64_t M, int64_t N, int64_t K) {
+  Plan p;
+  p.bt = pick_bt(M);
+  p.tiles_n = (int)((N + 127) / 128);
+  p.tiles_m = (int)((M + p.bt - 1) / p.bt);
+  const int64_t tiles = (int64_t)p.tiles_n * p.tiles_m;
+  const int G = (int)(K / 128);
+  const int64_t slots = (int64_t)dev_info().sms * ctas_per_sm(p.bt);
+  if (tiles < slots) {
+    int s = (int)(slots / tiles);
+    const int min_groups = 4;
+    s = s < G / min_groups ? s : G / min_groups;
+    p.splits = s > 1 ? s : 1;
+  }
+  return p;
+}
+
+size_t counters_bytes(const Plan& p) {
+  return (((size_t)p.tiles_n * p.tiles_m * 4) + 255) & ~(size_t)255;
+}
+
+size_t workspace_for(const Plan& p, int64_t M, int64_t N) {
+  if (p.splits <= 1) return 0;
+  return counters_bytes(p) + (size_t)p.splits * (size_t)M * (size_t)N * 4;
+}
+
+apex_status_t check_gemm_args(int64_t M, int64_t N, int64_t K, int32_t ga, int32_t gw) {
+  if (M <= 0 || N <= 0 || K <= 0) return APEX_ERR_INVALID_ARG;
+  if (ga <= 0 || gw <= 0 || K % ga || K % gw) return APEX_ERR_INVALID_ARG;
+  if (ga != 128) return APEX_ERR_UNSUPPORTED;
+  if (gw % 128) return APEX_ERR_UNSUPPORTED;
+  if (K % 128) return APEX_ERR_INVALID_ARG;
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return APEX_ERR_UNSUPPORTED;
+  return APEX_OK;
+}
+
+template <int BT, bool DUMP>
+apex_status_t launch_bt(const Plan& p, const CUtensorMap& tw, const CUtensorMap& ta,
+                        const GemmArgs& a, cudaStream_t s) {
+  using C = GemmCfg<BT>;
+  auto kern = apex::w4a4_gemm_kernel<BT, DUMP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return APEX_ERR_CUDA;
+  dim3 grid(p.tiles_n, p.tiles_m, a.splits);
+  kern<<<grid, C::THREADS, C::SMEM, s>>>(tw, ta, a);
+  return cuda_status(cudaPeekAtLastError());
+}
+
+template <bool DUMP>
+apex_status_t launch_gemm(const Plan& p, const CUtensorMap& tw, const CUtensorMap& ta,
+                          const GemmArgs& a, cudaStream_t s) {
+  switch (p.bt) {
+    case 16: return launch_bt<16, DUMP>(p, tw, ta, a, s);
+    case 32: return launch_bt<32, DUMP>(p, tw, ta, a, s);
+    case 64: return launch_bt<64, DUMP>(p, tw, ta, a, s);
+    default: return launch_bt<128, DUMP>(p, tw, ta, a, s);
+  }
+}
+
+apex_status_t quantize_launch(const void* x, int64_t rows, int64_t K, int32_t group, void* packed,
+                              void* scales, void* stream) {
+  if (!x || !packed || !scales) return APEX_ERR_INVALID_ARG;
+  if (rows <= 0 || K <= 0 || group <= 0 || K % group || group % 128) return APEX_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(packed, 4) || !aligned(scales, 2)) return APEX_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t units = rows * (K / group);
+  const int threads = 256;
+  const int64_t warps_needed = (units + 1) / 2;
+  int64_t blocks = (warps_needed * 32 + threads - 1) / threads;
+  const int64_t cap = (int64_t)dev_info().sms * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  const __half* xh = static_cast<const __half*>(x);
+  uint8_t* pk = static_cast<uint8_t*>(packed);
+  __half* sc = static_cast<__half*>(scales);
+  if (group == 128)
+    apex::quantize_pack_kernel<1><<<(unsigned)blocks, threads, 0, s>>>(xh, rows, K, group, pk, sc);
+  else if (group == 256)
+    apex::quantize_pack_kernel<2><<<(unsigned)blocks, threads, 0, s>>>(xh, rows, K, group, pk, sc);
+  else if (group == 512)
+    apex::quantize_pack_kernel<4><<<(unsigned)blocks, threads, 0, s>>>(xh, rows, K, group, pk, sc);
+  else
+    apex::quantize_pack_kernel<0><<<(unsigned)blocks, threads, 0, s>>>(xh, rows, K, group, pk, sc);
+  return cuda_status(cudaPeekAtLastError());
+}
+
+}  // namespace
+
+extern "C" {
+
+apex_status_t apex_pack_weights_int4(const void* w_f16, int64_t N, int64_t K, int32_t group_w,
+                                     void* w_packed_u8, void* w_scales_f16, void* stream) {
+  return quantize_launch(w_f16, N, K, group_w, w_packed_u8, w_scales_f16, stream);
+}
+
+apex_status_t apex_quantize_act_int4(const void* x_f16, int64_t M, int64_t K, int32_t group_a,
+                                     void* x_packed_u8, void* x_scales_f16, void* stream) {
+  return quantize_launch(x_f16, M, K, group_a, x_packed_u8, x_scales_f16, stream);
+}
+
+size_t apex_w4a4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                     int32_t group_w) {
+  if (check_gemm_args(M, N, K, group_a, group_w) != APEX_OK) return 0;
+  return workspace_for(make_plan(M, N, K), M, N);
+}
+
+apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, int32_t group_w,
+                             const void* a_packed, const void* a_scales, const void* w_packed,
+                             const void* w_scales, void* y_f16, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  apex_status_t st = check_gemm_args(M, N, K, group_a, group_w);
+  if (st != APEX_OK) return st;
+  if (!a_packed || !a_scales || !w_packed || !w_scales || !y_f16) return APEX_ERR_INVALID_ARG;
+  if (!aligned(a_packed, 16) || !aligned(w_packed, 16) || !aligned(a_scales, 2) ||
+      !aligned(w_scales, 2) || !aligned(y_f16, 2) || (workspace && !aligned(workspace, 256)))
+    return APEX_ERR_ALIGNMENT;
+
+  Plan p = make_plan(M, N, K);
+  // Shrink the split to what the caller's workspace holds.
+  while (p.splits > 1 && (!workspace || workspace_for(p, M, N) > workspace_bytes)) --p.splits;
+  const int G = (int)(K / 128);
+  GemmArgs a{};
+  a.M = (int)M;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.gw = group_w;
+  a.G = G;
+  a.Gw = (int)(K / group_w);
+  a.gps = (G + p.splits - 1) / p.splits;
+  a.splits = (G + a.gps - 1) / a.gps;  // no empty split
+  p.splits = a.splits;
+  a.sa = static_cast<const __half*>(a_scales);
+  a.sw = static_cast<const __half*>(w_scales);
+  a.y = static_cast<__half*>(y_f16);
+  if (p.splits > 1) {
+    a.counters = static_cast<unsigned*>(workspace);
+    a.ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + counters_bytes(p));
+  }
+  a.dump = nullptr;
+  a.wait_ns = g_wait_limit_ns;
+  a.withhold = t_withhold;
+  t_withhold = -1;
+
+  CUtensorMap tw, ta;
+  if (!make_packed_map(&tw, w_packed, N, K, 128) || !make_packed_map(&ta, a_packed, M, K, p.bt))
+    return APEX_ERR_CUDA;
+  return launch_gemm<false>(p, tw, ta, a, static_cast<cudaStream_t>(stream));
+}
+
+apex_status_t apex_w4a4_group_partials(int64_t M, int64_t N, int64_t K, const void* a_packed,
+                                       const void* w_packed, int32_t* partials_i32,
+                                       void* stream) {
+  apex_status_t st = check_gemm_args(M, N, K, 128, 128);
+  if (st != APEX_OK) return st;
+  if (!a_packed || !w_packed || !partials_i32) return APEX_ERR_INVALID_ARG;
+  if (!aligned(a_packed, 16) || !aligned(w_packed, 16) || !aligned(partials_i32, 4))
+    return APEX_ERR_ALIGNMENT;
+  Plan p = make_plan(M, N, K);
+  p.splits = 1;
+  GemmArgs a{};
+  a.M = (int)M;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.gw = 128;
+  a.G = (int)(K / 128);
+  a.Gw = a.G;
+  a.gps = a.G;
+  a.splits = 1;
+  a.dump = partials_i32;
+  a.wait_ns = g_wait_limit_ns;
+  a.withhold = -1;
+  CUtensorMap tw, ta;
+  if (!make_packed_map(&tw, w_packed, N, K, 128) || !make_packed_map(&ta, a_packed, M, K, p.bt))
+    return APEX_ERR_CUDA;
+  return launch_gemm<true>(p, tw, ta, a, static_cast<cudaStream_t>(stream));
+}
+
+apex_status_t apex_get_device_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return APEX_ERR_CUDA;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, apex::g_device_status, sizeof(v)) != cudaSuccess)
+    return APEX_ERR_CUDA;
+  if (v && cudaMemcpyToSymbol(apex::g_device_status, &zero, sizeof(zero)) != cudaSuccess)
+    return APEX_ERR_CUDA;
+  if (v & apex::DEV_TIMEOUT) return APEX_ERR_TIMEOUT;
+  return APEX_OK;
+}
+
+void apex_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns ? ns : 1; }
+
+void apex_debug_withhold_step(int32_t step) { t_withhold = step; }
+
+const char* apex_status_string(apex_status_t status) {
+  switch (status) {
+    case APEX_OK: return "ok";
+    case APEX_ERR_INVALID_ARG: return "invalid argument";
+    case APEX_ERR_UNSUPPORTED: return "unsupported configuration";
+    case APEX_ERR_ALIGNMENT: return "misaligned pointer";
+    case APEX_ERR_CUDA: return "CUDA error";
+    case APEX_ERR_TIMEOUT: return "device pipeline wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,123 @@
+/*
+ * apex_w4a4.h -- C ABI of the B200 (sm_100a) pure W4A4 group-quantized GEMM library.
+ *
+ * The operation: "APEX4: Efficient Pure W4A4 LLM Inference via Intra-SM Compute
+ * Rebalancing" (abstract) -- both GEMM operands are 4-bit integers with one fp16 scale per
+ * 128-wide K-group (the "W4A4-g128 kernel"); the INT4 tensor-core products of each group
+ * are dequantised with the group scales and summed.  Its "mixed-granularity mode" keeps
+ * 128-wide activation groups and uses coarser weight groups (here 512, or the whole row).
+ *
+ *   Y[m,n] = sum_g ( sum_{k in group g} qa[m,k] * qw[n,k] ) * sa[m,g] * sw[n, g*128/gw]
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library never
+ *     allocates device memory.
+ *   - Layouts are row-major with K contiguous.  Packed int4 rows: byte j of a row holds
+ *     element k = 2j in bits 0..3 and k = 2j+1 in bits 4..7, as two's-complement nibbles.
+ *     Scales are IEEE fp16, one per (row, group), row-major [rows][K/group].
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Every call
+ *     only enqueues work: it returns once the kernels are launched.
+ *   - Argument errors are detected on the host before anything is launched; nothing is
+ *     enqueued and the call returns APEX_ERR_INVALID_ARG / _UNSUPPORTED / _ALIGNMENT.
+ *     A failed launch returns APEX_ERR_CUDA.  Device-side problems (a pipeline wait that
+ *     ran out of time) are recorded in a status word read by apex_get_device_status().
+ */
+#ifndef APEX_W4A4_H
+#define APEX_W4A4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  APEX_OK = 0,
+  APEX_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, K not a multiple of group */
+  APEX_ERR_UNSUPPORTED = 2,  /* a group configuration this build does not implement */
+  APEX_ERR_ALIGNMENT = 3,    /* a pointer without the alignment stated for it */
+  APEX_ERR_CUDA = 4,         /* a CUDA runtime error (launch failure, no device, ...) */
+  APEX_ERR_TIMEOUT = 5       /* a device-side pipeline wait gave up (see apex_get_device_status) */
+} apex_status_t;
+
+/*
+ * Offline weight quantization and packing (per row, per K-group, symmetric).
+ * Rule (the plainest reading of the method's "W4", with fp16 scales):
+ *   s = fp16_rne(fp32(max_k |w[n,k]|) / 7)  (IEEE fp32 division),
+ *   q = clamp(round_half_even(fp32(w) / fp32(s)), -8, 7), q = 0 when s == 0.
+ *   w_f16        [N][K] fp16 (read)
+ *   w_packed_u8  [N][K/2] bytes (written)
+ *   w_scales_f16 [N][K/group_w] fp16 (written)
+ * group_w: a multiple of 128 that divides K (128, 512, ..., K).  K % 128 == 0.
+ * Alignment: w_f16 16 bytes, w_packed_u8 4 bytes, w_scales_f16 2 bytes.
+ */
+apex_status_t apex_pack_weights_int4(const void *w_f16, int64_t N, int64_t K, int32_t group_w,
+                                     void *w_packed_u8, void *w_scales_f16, void *stream);
+
+/*
+ * Online per-token, per-group activation quantization and packing: the same rule as
+ * apex_pack_weights_int4, applied to x_f16 [M][K] with group_a (128 for the GEMM).
+ *   x_packed_u8 [M][K/2], x_scales_f16 [M][K/group_a].
+ */
+apex_status_t apex_quantize_act_int4(const void *x_f16, int64_t M, int64_t K, int32_t group_a,
+                                     void *x_packed_u8, void *x_scales_f16, void *stream);
+
+/*
+ * The W4A4 GEMM: y_f16[M][N] = fp16_rne(sum_g P_g * sa * sw), accumulated in fp32.
+ *   a_packed [M][K/2], a_scales [M][K/group_a]   (from apex_quantize_act_int4)
+ *   w_packed [N][K/2], w_scales [N][K/group_w]   (from apex_pack_weights_int4)
+ * Supported: group_a == 128; group_w a multiple of 128 dividing K; K % 128 == 0;
+ * M, N >= 1 (ragged tiles are handled).  a_packed / w_packed 16-byte aligned, scales and
+ * y 2-byte aligned.
+ * workspace: device scratch for split-K partial sums, may be NULL (then no split-K).
+ *   Its size should be apex_w4a4_gemm_workspace_size(...); a smaller one limits the
+ *   split.  Its first bytes hold per-tile arrival counters that must be zero before the
+ *   first use (e.g. cudaMemset); every call that completes leaves them zero again.  Calls
+ *   that share a workspace must not run concurrently.
+ */
+apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, int32_t group_w,
+                             const void *a_packed, const void *a_scales, const void *w_packed,
+                             const void *w_scales, void *y_f16, void *workspace,
+                             size_t workspace_bytes, void *stream);
+
+/* Workspace bytes apex_w4a4_gemm would use for this problem (0 when it needs none). */
+size_t apex_w4a4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                     int32_t group_w);
+
+/*
+ * Debug / parity export: the exact integer partial of every 128-wide K-group,
+ *   partials_i32[g][m][n] = sum_{k in group g} qa[m,k] * qw[n,k],  g < K/128,
+ * computed by the same tensor-core path as apex_w4a4_gemm (its epilogue replaced by a
+ * store).  Same operand rules as apex_w4a4_gemm; partials_i32 4-byte aligned.
+ */
+apex_status_t apex_w4a4_group_partials(int64_t M, int64_t N, int64_t K, const void *a_packed,
+                                       const void *w_packed, int32_t *partials_i32,
+                                       void *stream);
+
+/*
+ * Synchronizes `stream`, then reads and clears the library's device status word.
+ * Returns APEX_ERR_TIMEOUT if a kernel since the last call gave up waiting on its own
+ * pipeline (its outputs are then undefined and a split-K workspace must be re-zeroed),
+ * APEX_ERR_CUDA on a CUDA error, else APEX_OK.
+ */
+apex_status_t apex_get_device_status(void *stream);
+
+/* Time limit, in nanoseconds, of every device-side pipeline wait (default 2e9). */
+void apex_set_wait_limit_ns(uint64_t ns);
+
+/* Static description of a status code (never NULL). */
+const char *apex_status_string(apex_status_t status);
+
+/*
+ * Test hook: the next GEMM launch on this host thread skips the bulk copy of K-group step
+ * `step` (counted within each CTA), so its consumers wait until the time limit.  -1 turns
+ * it off.  Used only to test the timeout path; never needed by callers.
+ */
+void apex_debug_withhold_step(int32_t step);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* APEX_W4A4_H */

@@ -1,0 +1,106 @@
+"""CPU checks of the C-ABI library: it builds for sm_100a, loads, exports every entry point
+that include/apex_w4a4.h declares, and rejects bad arguments on the host before touching
+the GPU.  No compute call runs here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import group_quantized_w4a4_b200 as apex
+from group_quantized_w4a4_b200 import build as apex_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "apex_w4a4.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(apex_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    apex_build.build()
+    return apex.load_library()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("apex_pack_weights_int4", "apex_quantize_act_int4", "apex_w4a4_gemm",
+                 "apex_w4a4_gemm_workspace_size", "apex_w4a4_group_partials",
+                 "apex_get_device_status", "apex_status_string"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert getattr(apex, name, None) is not None, f"binding lacks {name}"
+
+
+def test_library_is_sm100a_only():
+    assert apex_build.ARCH_FLAGS == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert apex.apex_status_string(code)
+    assert apex.apex_status_string(5) == "device pipeline wait timed out"
+
+
+P = ctypes.c_void_p
+
+
+def _gemm(lib, M, N, K, ga, gw, a=0x1000, sa=0x2000, w=0x3000, sw=0x4000, y=0x5000,
+          ws=None, wsb=0):
+    return lib.apex_w4a4_gemm(M, N, K, ga, gw, P(a), P(sa), P(w), P(sw), P(y),
+                              P(ws) if ws else None, wsb, None)
+
+
+def test_gemm_argument_errors_are_host_side(lib):
+    assert _gemm(lib, 0, 8, 128, 128, 128) == apex.APEX_ERR_INVALID_ARG
+    assert _gemm(lib, 4, -1, 128, 128, 128) == apex.APEX_ERR_INVALID_ARG
+    assert _gemm(lib, 4, 8, 100, 128, 128) == apex.APEX_ERR_INVALID_ARG      # K % ga
+    assert _gemm(lib, 4, 8, 256, 128, 96) == apex.APEX_ERR_INVALID_ARG       # K % gw
+    assert _gemm(lib, 4, 8, 512, 256, 256) == apex.APEX_ERR_UNSUPPORTED      # ga != 128
+    assert _gemm(lib, 4, 8, 192, 64, 192) == apex.APEX_ERR_UNSUPPORTED
+    assert _gemm(lib, 4, 8, 256, 128, 128, a=0) == apex.APEX_ERR_INVALID_ARG  # null
+    assert _gemm(lib, 4, 8, 256, 128, 128, a=0x1008) == apex.APEX_ERR_ALIGNMENT
+    assert _gemm(lib, 4, 8, 256, 128, 128, w=0x3004) == apex.APEX_ERR_ALIGNMENT
+    assert _gemm(lib, 4, 8, 256, 128, 128, y=0x5001) == apex.APEX_ERR_ALIGNMENT
+
+
+def test_quantizer_argument_errors_are_host_side(lib):
+    q = lib.apex_quantize_act_int4
+    assert q(None, 4, 256, 128, P(0x1000), P(0x2000), None) == apex.APEX_ERR_INVALID_ARG
+    assert q(P(0x1000), 4, 200, 128, P(0x2000), P(0x3000), None) == apex.APEX_ERR_INVALID_ARG
+    assert q(P(0x1000), 4, 256, 64, P(0x2000), P(0x3000), None) == apex.APEX_ERR_INVALID_ARG
+    assert q(P(0x1008), 4, 256, 128, P(0x2000), P(0x3000), None) == apex.APEX_ERR_ALIGNMENT
+    pw = lib.apex_pack_weights_int4
+    assert pw(P(0x1000), 0, 256, 128, P(0x2000), P(0x3000), None) == apex.APEX_ERR_INVALID_ARG
+    assert pw(P(0x1000), 4, 256, 128, P(0x2002), P(0x3000), None) == apex.APEX_ERR_ALIGNMENT
+
+
+def test_partials_argument_errors(lib):
+    f = lib.apex_w4a4_group_partials
+    assert f(4, 8, 100, P(0x1000), P(0x2000), P(0x3000), None) == apex.APEX_ERR_INVALID_ARG
+    assert f(4, 8, 256, P(0x1000), P(0x2000), None, None) == apex.APEX_ERR_INVALID_ARG
+    assert f(4, 8, 256, P(0x1001), P(0x2000), P(0x3000), None) == apex.APEX_ERR_ALIGNMENT
+
+
+def test_workspace_size_contract(lib):
+    # invalid problems need no workspace; a decode-shaped problem uses split-K scratch
+    assert lib.apex_w4a4_gemm_workspace_size(0, 8, 128, 128, 128) == 0
+    n = lib.apex_w4a4_gemm_workspace_size(16, 8192, 8192, 128, 128)
+    assert n == 0 or n >= 16 * 8192 * 4 * 2
+    # a prefill-shaped problem has enough tiles to fill the GPU without splitting K
+    assert lib.apex_w4a4_gemm_workspace_size(4096, 8192, 8192, 128, 128) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros((4, 256), dtype=torch.float16)
+    with pytest.raises((ValueError, RuntimeError)):
+        apex.quantize_act(x)

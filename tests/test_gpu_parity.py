@@ -1,0 +1,295 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Bars (the method: "APEX4: Efficient Pure W4A4 LLM Inference via Intra-SM Compute
+Rebalancing", abstract -- W4A4 with per-128-group scales, INT4 products dequantised per
+group):
+  * packed int4 operands and fp16 scales: bit-exact;
+  * per-group integer partials: bit-exact;
+  * fp16 output: |y - y_ref| <= 2^-10 |y_ref| + 1e-3 max|y_ref| against the fp64 oracle.
+Inputs are the seeded synthetic workloads of group_quantized_w4a4_b200.synth.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from group_quantized_w4a4_b200 import synth
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def apex():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import group_quantized_w4a4_b200 as m
+    m.load_library()
+    return m
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    return t.cpu().numpy()
+
+
+def f16(t):
+    return host(t).view(np.uint16)
+
+
+def check_status(apex):
+    assert apex.apex_get_device_status() == 0
+
+
+# ------------------------------------------------------------------ quantizer
+
+
+@pytest.mark.parametrize("rows,K,dist", [(16, 512, "normal"), (37, 1024, "outlier"),
+                                         (129, 2048, "student_t"), (1, 128, "normal")])
+def test_quantize_act_bit_exact(apex, rows, K, dist):
+    x = synth.activations(rows, K, dist, 7 + rows)
+    ap_ref, sa_ref = oracle.quantize_pack(x, 128)
+    ap, sa = apex.quantize_act(dev(x), 128)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(ap), ap_ref)
+    assert np.array_equal(f16(sa), sa_ref.view(np.uint16))
+    check_status(apex)
+
+
+@pytest.mark.parametrize("group", [128, 256, 512, 1024, 3072])
+def test_pack_weights_bit_exact(apex, group):
+    K = 3072
+    w = synth.weights(70, K, 11)
+    wp_ref, sw_ref = oracle.quantize_pack(w, group)
+    wp, sw = apex.pack_weights(dev(w), group)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(wp), wp_ref)
+    assert np.array_equal(f16(sw), sw_ref.view(np.uint16))
+
+
+def test_quantize_edge_values(apex):
+    rng = np.random.default_rng(5)
+    K = 512
+    x = np.zeros((6, K), dtype=np.float16)
+    x[1, :128] = 7.0
+    x[1, 1:14] = [0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.5, 4.5, 5.5, 6.5, -6.5, 0.25, 0.75]
+    x[2] = (rng.integers(-7, 8, K) * 0.5).astype(np.float16)          # many ties
+    x[3] = (rng.standard_normal(K) * 1e-5).astype(np.float16)         # subnormal scales
+    x[4, 128:256] = np.float16(2.0 ** -24)                              # scale underflows
+    x[5] = (rng.standard_normal(K) * 3000).astype(np.float16)          # large values
+    ap_ref, sa_ref = oracle.quantize_pack(x, 128)
+    ap, sa = apex.quantize_act(dev(x), 128)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(ap), ap_ref)
+    assert np.array_equal(f16(sa), sa_ref.view(np.uint16))
+
+
+def test_quantize_full_size_bit_exact(apex):
+    g = synth.workloads()["prefill_m4096_n8192_k8192"]
+    x = synth.activations(g.M, g.K, g.act, g.seed)
+    ap_ref, sa_ref = oracle.quantize_pack(x, 128)
+    ap, sa = apex.quantize_act(dev(x), 128)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(ap), ap_ref)
+    assert np.array_equal(f16(sa), sa_ref.view(np.uint16))
+
+
+# ------------------------------------------------------------------ integer partials
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 256, 512), (1, 128, 128), (17, 200, 384),
+                                   (64, 128, 256), (100, 384, 640), (129, 130, 256),
+                                   (256, 256, 1024)])
+def test_group_partials_bit_exact_random_bytes(apex, M, N, K):
+    rng = np.random.default_rng(M * 7 + N + K)
+    ap = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)   # includes -8 nibbles
+    wp = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    ref = oracle.group_partials(ap, wp, M, N, K, 128, 128)
+    out = torch.empty((K // 128, M, N), dtype=torch.int32, device="cuda")
+    apex.apex_w4a4_group_partials(M, N, K, dev(ap), dev(wp), out)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(out).astype(np.int64), ref)
+    check_status(apex)
+
+
+def test_group_partials_extremes(apex):
+    M, N, K = 16, 128, 256
+    ap = np.full((M, K // 2), 0x88, dtype=np.uint8)                     # all -8
+    wp = np.full((N, K // 2), 0x88, dtype=np.uint8)
+    wp[1::2] = 0x77                                                     # all +7
+    ref = oracle.group_partials(ap, wp, M, N, K, 128, 128)
+    out = torch.empty((K // 128, M, N), dtype=torch.int32, device="cuda")
+    apex.apex_w4a4_group_partials(M, N, K, dev(ap), dev(wp), out)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(out).astype(np.int64), ref)
+    assert ref.max() == 128 * 64 and ref.min() == -128 * 56
+
+
+def test_group_partials_quantized_workload(apex):
+    g = synth.workloads()["tiny_m16_n256_k512"]
+    a, w = synth.make(g)
+    ap, _ = oracle.quantize_pack(a, 128)
+    wp, _ = oracle.quantize_pack(w, 128)
+    ref = oracle.group_partials(ap, wp, g.M, g.N, g.K, 128, 128)
+    out = torch.empty((g.K // 128, g.M, g.N), dtype=torch.int32, device="cuda")
+    apex.apex_w4a4_group_partials(g.M, g.N, g.K, dev(ap), dev(wp), out)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(out).astype(np.int64), ref)
+
+
+# ------------------------------------------------------------------ GEMM output
+
+
+def run_gemm(apex, ap, sa, wp, sw, M, N, K, gw, ws=True):
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    w = apex.workspace(M, N, K, 128, gw) if ws else None
+    apex.apex_w4a4_gemm(M, N, K, 128, gw, dev(ap), dev(sa), dev(wp), dev(sw), y, w)
+    torch.cuda.synchronize()
+    check_status(apex)
+    return host(y).astype(np.float64)
+
+
+def assert_close(y, ref, max_abs_ref=None):
+    ok, ratio = oracle.within_tolerance(y, ref, max_abs_ref)
+    assert ok, f"tolerance exceeded: worst err/bound = {ratio:.3f}"
+
+
+@pytest.mark.parametrize("M,N,K,gw", [
+    (16, 256, 512, 128), (1, 128, 128, 128), (15, 200, 384, 128), (17, 300, 1024, 512),
+    (33, 128, 512, 512), (64, 256, 1024, 1024), (65, 129, 640, 128), (129, 257, 768, 768),
+    (200, 384, 2048, 128), (256, 128, 1024, 256)])
+def test_gemm_matches_oracle(apex, M, N, K, gw):
+    a = synth.activations(M, K, "outlier", M + K)
+    w = synth.weights(N, K, N + K)
+    ap, sa = oracle.quantize_pack(a, 128)
+    wp, sw = oracle.quantize_pack(w, gw)
+    ref = oracle.gemm(ap, sa, wp, sw, M, N, K, 128, gw)
+    assert_close(run_gemm(apex, ap, sa, wp, sw, M, N, K, gw), ref)
+
+
+def test_gemm_without_workspace_matches(apex):
+    M, N, K = 16, 1024, 4096
+    a = synth.activations(M, K, "normal", 3)
+    w = synth.weights(N, K, 3)
+    ap, sa = oracle.quantize_pack(a, 128)
+    wp, sw = oracle.quantize_pack(w, 128)
+    ref = oracle.gemm(ap, sa, wp, sw, M, N, K, 128, 128)
+    assert_close(run_gemm(apex, ap, sa, wp, sw, M, N, K, 128, ws=False), ref)
+    assert_close(run_gemm(apex, ap, sa, wp, sw, M, N, K, 128, ws=True), ref)
+
+
+def test_gemm_random_bytes_and_scales(apex):
+    rng = np.random.default_rng(99)
+    M, N, K = 48, 256, 1024
+    ap = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    wp = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    sa = rng.uniform(0.01, 4.0, size=(M, K // 128)).astype(np.float16)
+    sw = rng.uniform(1e-4, 0.05, size=(N, K // 128)).astype(np.float16)
+    ref = oracle.gemm(ap, sa, wp, sw, M, N, K, 128, 128)
+    assert_close(run_gemm(apex, ap, sa, wp, sw, M, N, K, 128), ref)
+
+
+def test_gemm_split_k_is_deterministic(apex):
+    M, N, K = 16, 2048, 8192
+    a = synth.activations(M, K, "normal", 1)
+    w = synth.weights(N, K, 1)
+    ap, sa = oracle.quantize_pack(a, 128)
+    wp, sw = oracle.quantize_pack(w, 128)
+    ws = apex.workspace(M, N, K)
+    assert ws is not None
+    args = [dev(x) for x in (ap, sa, wp, sw)]
+    outs = []
+    for _ in range(3):
+        y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+        apex.apex_w4a4_gemm(M, N, K, 128, 128, *args, y, ws)
+        outs.append(y)
+    torch.cuda.synchronize()
+    assert all(torch.equal(outs[0], o) for o in outs[1:])
+    assert int(ws[:256].sum()) == 0        # arrival counters are left at zero
+
+
+def test_gemm_scale_linearity(apex):
+    M, N, K = 32, 256, 1024
+    a = synth.activations(M, K, "normal", 8)
+    w = synth.weights(N, K, 8)
+    ap, sa = oracle.quantize_pack(a, 128)
+    wp, sw = oracle.quantize_pack(w, 128)
+    y0 = run_gemm(apex, ap, sa, wp, sw, M, N, K, 128)
+    sw2 = sw.copy()
+    sw2[5] = (sw2[5].astype(np.float32) * 2).astype(np.float16)
+    y1 = run_gemm(apex, ap, sa, wp, sw2, M, N, K, 128)
+    want = y0.copy()
+    want[:, 5] *= 2
+    assert np.array_equal(y1, want)
+
+
+@pytest.mark.parametrize("name", ["tiny_m16_n256_k512", "decode_m16_n8192_k8192"])
+def test_gemm_full_workloads(apex, name):
+    g = synth.workloads()[name]
+    a, w = synth.make(g)
+    ap, sa = oracle.quantize_pack(a, 128)
+    wp, sw = oracle.quantize_pack(w, g.gw)
+    ref = oracle.gemm(ap, sa, wp, sw, g.M, g.N, g.K, 128, g.gw)
+    assert_close(run_gemm(apex, ap, sa, wp, sw, g.M, g.N, g.K, g.gw), ref)
+
+
+SAMPLED = ["prefill_m4096_n8192_k8192", "mlp_up_m2048_n28672_k8192",
+           "mlp_down_m2048_n8192_k28672", "sweep_m1_gw128", "sweep_m128_gw512",
+           "sweep_m1024_gw8192", "sweep_m4096_gw512", "sweep_m16_gw8192"]
+
+
+@pytest.mark.parametrize("name", SAMPLED)
+def test_gemm_large_workloads_sampled_rows(apex, name):
+    """Full-size problem in the benchmark's launch configuration; the whole pipeline
+    (quantizer + GEMM) runs on the GPU, the oracle checks sampled output rows."""
+    g = synth.workloads()[name]
+    a, w = synth.make(g)
+    a_d, w_d = dev(a), dev(w)
+    ap, sa = apex.quantize_act(a_d, 128)
+    wp, sw = apex.pack_weights(w_d, g.gw)
+    ws = apex.workspace(g.M, g.N, g.K, 128, g.gw)
+    y = apex.gemm(ap, sa, wp, sw, 128, g.gw, ws=ws)
+    torch.cuda.synchronize()
+    check_status(apex)
+    rng = np.random.default_rng(0)
+    cand = {0, g.M - 1, min(127, g.M - 1), min(128, g.M - 1), g.M // 2}
+    cand |= set(rng.integers(0, g.M, size=min(g.M, 12)).tolist())
+    rows = np.array(sorted(cand), dtype=np.int64)
+    ap_h, sa_h, wp_h, sw_h = host(ap), host(sa), host(wp), host(sw)
+    # the GPU-packed operands are themselves checked against the oracle's quantizer
+    ap_ref, sa_ref = oracle.quantize_pack(a[rows], 128)
+    assert np.array_equal(ap_h[rows], ap_ref)
+    assert np.array_equal(sa_h[rows].view(np.uint16), sa_ref.view(np.uint16))
+    wrows = np.array(sorted({0, g.N - 1, 4097 % g.N, 77}), dtype=np.int64)
+    wp_ref, sw_ref = oracle.quantize_pack(w[wrows], g.gw)
+    assert np.array_equal(wp_h[wrows], wp_ref)
+    assert np.array_equal(sw_h[wrows].view(np.uint16), sw_ref.view(np.uint16))
+    ref = oracle.gemm(ap_h, sa_h, wp_h, sw_h, g.M, g.N, g.K, 128, g.gw, rows=rows)
+    got = host(y)[rows].astype(np.float64)
+    # max|ref| over the whole output is at least the sampled max: using the sampled max
+    # makes the absolute term of the bound no looser than the stated rule.
+    assert_close(got, ref)
+
+
+# ------------------------------------------------------------------ failure path
+
+
+def test_pipeline_wait_timeout_is_reported_and_context_survives(apex):
+    M, N, K = 16, 256, 1024
+    a = synth.activations(M, K, "normal", 2)
+    w = synth.weights(N, K, 2)
+    ap, sa = oracle.quantize_pack(a, 128)
+    wp, sw = oracle.quantize_pack(w, 128)
+    args = [dev(x) for x in (ap, sa, wp, sw)]
+    y = torch.zeros((M, N), dtype=torch.float16, device="cuda")
+    apex.apex_set_wait_limit_ns(50_000_000)           # 50 ms
+    try:
+        apex.apex_debug_withhold_step(1)              # one bulk copy never issued
+        apex.apex_w4a4_gemm(M, N, K, 128, 128, *args, y, None)
+        assert apex.apex_get_device_status() == apex.APEX_ERR_TIMEOUT
+    finally:
+        apex.apex_set_wait_limit_ns(2_000_000_000)
+    ref = oracle.gemm(ap, sa, wp, sw, M, N, K, 128, 128)
+    assert_close(run_gemm(apex, ap, sa, wp, sw, M, N, K, 128), ref)
