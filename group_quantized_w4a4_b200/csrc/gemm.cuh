@@ -267,11 +267,14 @@ __global__ void __launch_bounds__(GemmCfg<BT>::THREADS, GemmCfg<BT>::MIN_BLOCKS)
     constexpr int NE = C::EPI_WARPS * 32;
     const int M = args.M, N = args.N;
 
+    // The partials export has no scales (its launch passes none): never touch them there.
     auto load_sa = [&](int g) -> float {
+      if constexpr (DUMP) return 0.0f;
       const int m = m0 + et;
       return (et < BT && m < M) ? __half2float(args.sa[(size_t)m * args.G + g]) : 0.0f;
     };
     auto load_sw = [&](int g) -> float {
+      if constexpr (DUMP) return 0.0f;
       return nvalid ? __half2float(args.sw[(size_t)n * args.Gw + (g * 128) / args.gw]) *
                           (1.0f / 256.0f)
                     : 0.0f;
