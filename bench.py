@@ -18,7 +18,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -83,49 +82,69 @@ def max_over_ranks(x: float, world: int) -> float:
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Polls the SM clock and the clock-event (throttle) reasons through NVML from a
+    background thread while the timed region runs (read-only queries)."""
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = None
+        self._thread = None
+        self._err = None
+
+    def _handle(self, nv):
+        import torch
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.cuda_index).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-")
+                                                else uuid)
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            idx = int(vis.split(",")[self.cuda_index]) if vis and vis.split(",")[0].isdigit() \
+                else self.cuda_index
+            return nv.nvmlDeviceGetHandleByIndex(idx)
 
     def start(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception as e:  # no NVML: report that instead of clocks
+            self._err = f"nvml unavailable: {type(e).__name__}"
+            return
+        self._stop = threading.Event()
+
+        def poll():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    self.reasons |= int(get_reasons(h))
+                except Exception:
+                    pass
+                self._stop.wait(0.002)
+
+        self._thread = threading.Thread(target=poll, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        if self._thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0,
+                    "reasons": [self._err or "not sampled"]}
+        self._stop.set()
+        self._thread.join(timeout=2)
+        names = sorted(v for k, v in self.REASONS.items() if self.reasons & k)
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples), "reasons": names,
+                "source": "NVML polled every 2 ms during the timed region"}
 
 
 # ------------------------------------------------------------------ the apex arm
@@ -166,42 +185,56 @@ def copies_for(g: synth.Gemm, l2_bytes: int) -> int:
 def apex_step(apex, p: Problem, i: int, stream, ev=None):
     g = p.g
     c = i % p.copies
-    apex.apex_quantize_act_int4(p.x[c], g.M, g.K, 128, p.ap[c], p.sa[c], stream)
     if ev is not None:
         ev[0].record(stream)
+    apex.apex_quantize_act_int4(p.x[c], g.M, g.K, 128, p.ap[c], p.sa[c], stream)
+    if ev is not None:
+        ev[1].record(stream)
     apex.apex_w4a4_gemm(g.M, g.N, g.K, 128, g.gw, p.ap[c], p.sa[c], p.wp[c], p.sw[c], p.y,
                         p.ws, None, stream)
     if ev is not None:
-        ev[1].record(stream)
+        ev[2].record(stream)
 
 
 def time_workload(apex, torch, g, steps, warmup, world, l2_bytes, clocks=None):
+    """W eager warm-up steps, then exactly K steps replayed from one CUDA graph (captured
+    beforehand, so the timed region has no host launch overhead), CUDA events around
+    every kernel inside the graph."""
     p = Problem(apex, torch, g, copies_for(g, l2_bytes))
-    stream = torch.cuda.current_stream()
     for i in range(warmup):
-        apex_step(apex, p, i, stream)
+        apex_step(apex, p, i, torch.cuda.current_stream())
     torch.cuda.synchronize()
-    if apex.apex_get_device_status(stream) != 0:
+    if apex.apex_get_device_status() != 0:
         raise RuntimeError("device status not clean after warm-up")
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    # external=True: captured as real event-record nodes, so they time the replay
+    evs = [tuple(torch.cuda.Event(enable_timing=True, external=True) for _ in range(3))
            for _ in range(steps)]
+    side = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            for i in range(steps):
+                apex_step(apex, p, warmup + i, side, evs[i])
+    torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     if clocks:
         clocks.start()
-    start.record(stream)
-    for i in range(steps):
-        apex_step(apex, p, warmup + i, stream, evs[i])
-    stop.record(stream)
+    with torch.cuda.stream(side):
+        start.record(side)
+        graph.replay()
+        stop.record(side)
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop() if clocks else None
-    if apex.apex_get_device_status(stream) != 0:
+    if apex.apex_get_device_status() != 0:
         raise RuntimeError("device status not clean after the timed steps")
     total_ms = start.elapsed_time(stop)
-    gemm_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
-    return p, total_ms, gemm_ms, clk
+    quant_ms = [e0.elapsed_time(e1) for e0, e1, _ in evs]
+    gemm_ms = [e1.elapsed_time(e2) for _, e1, e2 in evs]
+    del graph
+    return p, total_ms, gemm_ms, clk, quant_ms
 
 
 def e2e_workload(apex, torch, g, steps, warmup, p: Problem):
@@ -289,8 +322,8 @@ def run_apex(args, rank, world, local):
     peaks, peaks_kind = load_peaks()
     g = synth.workloads()[args.workload]
     clocks = ClockSampler(local) if rank == 0 else None
-    p, total_ms, gemm_ms, clk = time_workload(apex, torch, g, args.steps, args.warmup, world,
-                                              l2, clocks)
+    p, total_ms, gemm_ms, clk, quant_ms = time_workload(apex, torch, g, args.steps,
+                                                        args.warmup, world, l2, clocks)
     ms_step = max_over_ranks(total_ms / args.steps, world)
     gemm_avg = statistics.mean(gemm_ms)
     value = world * g.ops / (ms_step * 1e-3) / 1e12
@@ -301,12 +334,13 @@ def run_apex(args, rank, world, local):
     extra = {}
     if not args.no_second and args.workload != SECOND_WORKLOAD:
         g2 = synth.workloads()[SECOND_WORKLOAD]
-        p2, tot2, gm2, _ = time_workload(apex, torch, g2, max(3, args.steps // 4),
-                                         args.warmup, world, l2)
+        p2, tot2, gm2, _, qm2 = time_workload(apex, torch, g2, max(3, args.steps // 4),
+                                              args.warmup, world, l2)
         ms2 = max_over_ranks(tot2 / max(3, args.steps // 4), world)
         extra[SECOND_WORKLOAD] = {
             "value": round(world * g2.ops / (ms2 * 1e-3) / 1e12, 2), "unit": "TOPS",
             "ms_per_step": round(ms2, 4),
+            "quantize_ms": round(statistics.mean(qm2), 5),
             "roofline": roofline_obj(g2, statistics.mean(gm2), peaks, peaks_kind)}
         del p2
     if rank != 0:
@@ -325,6 +359,11 @@ def run_apex(args, rank, world, local):
                 "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db,
                 "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": 2 * args.steps,
+        "launch": "one CUDA graph of the K timed steps (eager warm-up)",
+        "quantize": {"kernel_ms": round(statistics.mean(quant_ms), 5),
+                     "bytes": g.quant_bytes(),
+                     "GB/s": round(g.quant_bytes() / (statistics.mean(quant_ms) * 1e-3) / 1e9,
+                                   1)},
         "clocks": clk,
         "impl": "apex",
     }
@@ -366,7 +405,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.workloads()))
     ap.add_argument("--impl", default="apex", choices=["apex", "reference"])

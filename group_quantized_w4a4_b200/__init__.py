@@ -23,6 +23,7 @@ __all__ = [
     "apex_pack_weights_int4", "apex_quantize_act_int4", "apex_w4a4_gemm",
     "apex_w4a4_gemm_workspace_size", "apex_w4a4_group_partials", "apex_get_device_status",
     "apex_set_wait_limit_ns", "apex_status_string", "apex_debug_withhold_step",
+    "apex_debug_trace_next_gemm",
     "pack_weights", "quantize_act", "gemm", "workspace",
 ]
 
@@ -82,6 +83,8 @@ def load_library(build_if_missing: bool = True):
         lib.apex_status_string.restype = ctypes.c_char_p
         lib.apex_debug_withhold_step.argtypes = [I32]
         lib.apex_debug_withhold_step.restype = None
+        lib.apex_debug_trace_next_gemm.argtypes = [P, I32, I32]
+        lib.apex_debug_trace_next_gemm.restype = None
         _lib = lib
         return lib
 
@@ -162,6 +165,13 @@ def apex_set_wait_limit_ns(ns: int):
 
 def apex_debug_withhold_step(step: int):
     load_library().apex_debug_withhold_step(int(step))
+
+
+def apex_debug_trace_next_gemm(trace, ctas: int, steps: int):
+    """trace: int64 CUDA tensor with at least ctas*6*steps elements (zeroed by the caller)."""
+    if trace.numel() < ctas * 6 * steps:
+        raise ValueError("trace buffer too small")
+    load_library().apex_debug_trace_next_gemm(_ptr(trace), int(ctas), int(steps))
 
 
 # ------------------------------------------------------------------ tensor conveniences

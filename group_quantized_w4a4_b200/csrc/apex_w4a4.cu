@@ -22,6 +22,9 @@ using apex::GemmCfg;
 
 uint64_t g_wait_limit_ns = 2000000000ull;
 thread_local int t_withhold = -1;
+thread_local unsigned long long* t_trace = nullptr;
+thread_local int t_trace_ctas = 0;
+thread_local int t_trace_steps = 0;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -74,18 +77,33 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D map over a packed int4 matrix [rows][K/2] bytes; box = 64 bytes (one 128-wide
-// K-group) x box_rows rows, 64-byte swizzle, out-of-range rows read as zeros.
+// 2-D map over a packed int4 matrix [rows][K/2] bytes; box = 128 bytes (two 128-wide
+// K-groups) x box_rows rows, 128-byte swizzle; out-of-range rows and columns read as zeros.
 bool make_packed_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1u, 1u};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 2-D map over an fp16 scale matrix [rows][cols]; box = 8 columns (16 bytes) x box_rows.
+// Needs a 16-byte aligned base and cols % 8 == 0 (row stride a multiple of 16 bytes).
+bool make_scale_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
+  cuuint32_t box[2] = {8u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -142,27 +160,35 @@ apex_status_t check_gemm_args(int64_t M, int64_t N, int64_t K, int32_t ga, int32
   return APEX_OK;
 }
 
-template <int BT, bool DUMP>
-apex_status_t launch_bt(const Plan& p, const CUtensorMap& tw, const CUtensorMap& ta,
-                        const GemmArgs& a, cudaStream_t s) {
+struct Maps {
+  CUtensorMap w, a, sa, sw;
+};
+
+template <int BT, bool DUMP, bool SCT>
+apex_status_t launch_bt(const Plan& p, const Maps& m, const GemmArgs& a, cudaStream_t s) {
   using C = GemmCfg<BT>;
-  auto kern = apex::w4a4_gemm_kernel<BT, DUMP>;
+  auto kern = apex::w4a4_gemm_kernel<BT, DUMP, SCT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return APEX_ERR_CUDA;
   dim3 grid(p.tiles_n, p.tiles_m, a.splits);
-  kern<<<grid, C::THREADS, C::SMEM, s>>>(tw, ta, a);
+  kern<<<grid, C::THREADS, C::SMEM, s>>>(m.w, m.a, m.sa, m.sw, a);
   return cuda_status(cudaPeekAtLastError());
 }
 
-template <bool DUMP>
-apex_status_t launch_gemm(const Plan& p, const CUtensorMap& tw, const CUtensorMap& ta,
-                          const GemmArgs& a, cudaStream_t s) {
+template <bool DUMP, bool SCT>
+apex_status_t launch_gemm_sct(const Plan& p, const Maps& m, const GemmArgs& a, cudaStream_t s) {
   switch (p.bt) {
-    case 16: return launch_bt<16, DUMP>(p, tw, ta, a, s);
-    case 32: return launch_bt<32, DUMP>(p, tw, ta, a, s);
-    case 64: return launch_bt<64, DUMP>(p, tw, ta, a, s);
-    default: return launch_bt<128, DUMP>(p, tw, ta, a, s);
+    case 16: return launch_bt<16, DUMP, SCT>(p, m, a, s);
+    case 32: return launch_bt<32, DUMP, SCT>(p, m, a, s);
+    case 64: return launch_bt<64, DUMP, SCT>(p, m, a, s);
+    default: return launch_bt<128, DUMP, SCT>(p, m, a, s);
   }
+}
+
+template <bool DUMP>
+apex_status_t launch_gemm(const Plan& p, const Maps& m, const GemmArgs& a, bool sct,
+                          cudaStream_t s) {
+  return sct ? launch_gemm_sct<DUMP, true>(p, m, a, s) : launch_gemm_sct<DUMP, false>(p, m, a, s);
 }
 
 apex_status_t quantize_launch(const void* x, int64_t rows, int64_t K, int32_t group, void* packed,
@@ -227,14 +253,19 @@ apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, i
   // Shrink the split to what the caller's workspace holds.
   while (p.splits > 1 && (!workspace || workspace_for(p, M, N) > workspace_bytes)) --p.splits;
   const int G = (int)(K / 128);
+  const int Gw = (int)(K / group_w);
+  // Scales by TMA need 16-byte row strides and bases, and splits starting on 8-group blocks.
+  const bool sct = G % 8 == 0 && (Gw % 8 == 0 || Gw == 1) && aligned(a_scales, 16) &&
+                   aligned(w_scales, 16);
   GemmArgs a{};
   a.M = (int)M;
   a.N = (int)N;
   a.K = (int)K;
   a.gw = group_w;
   a.G = G;
-  a.Gw = (int)(K / group_w);
+  a.Gw = Gw;
   a.gps = (G + p.splits - 1) / p.splits;
+  if (sct) a.gps = (a.gps + 7) / 8 * 8;
   a.splits = (G + a.gps - 1) / a.gps;  // no empty split
   p.splits = a.splits;
   a.sa = static_cast<const __half*>(a_scales);
@@ -248,11 +279,21 @@ apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, i
   a.wait_ns = g_wait_limit_ns;
   a.withhold = t_withhold;
   t_withhold = -1;
+  a.trace = t_trace;
+  a.trace_ctas = t_trace_ctas;
+  a.trace_steps = t_trace_steps;
+  t_trace = nullptr;
 
-  CUtensorMap tw, ta;
-  if (!make_packed_map(&tw, w_packed, N, K, 128) || !make_packed_map(&ta, a_packed, M, K, p.bt))
+  Maps maps;
+  memset(&maps, 0, sizeof(maps));
+  if (!make_packed_map(&maps.w, w_packed, N, K, 128) ||
+      !make_packed_map(&maps.a, a_packed, M, K, p.bt))
     return APEX_ERR_CUDA;
-  return launch_gemm<false>(p, tw, ta, a, static_cast<cudaStream_t>(stream));
+  if (sct) {
+    if (!make_scale_map(&maps.sa, a_scales, M, G, p.bt)) return APEX_ERR_CUDA;
+    if (Gw % 8 == 0 && !make_scale_map(&maps.sw, w_scales, N, Gw, 128)) return APEX_ERR_CUDA;
+  }
+  return launch_gemm<false>(p, maps, a, sct, static_cast<cudaStream_t>(stream));
 }
 
 apex_status_t apex_w4a4_group_partials(int64_t M, int64_t N, int64_t K, const void* a_packed,
@@ -277,10 +318,12 @@ apex_status_t apex_w4a4_group_partials(int64_t M, int64_t N, int64_t K, const vo
   a.dump = partials_i32;
   a.wait_ns = g_wait_limit_ns;
   a.withhold = -1;
-  CUtensorMap tw, ta;
-  if (!make_packed_map(&tw, w_packed, N, K, 128) || !make_packed_map(&ta, a_packed, M, K, p.bt))
+  Maps maps;
+  memset(&maps, 0, sizeof(maps));
+  if (!make_packed_map(&maps.w, w_packed, N, K, 128) ||
+      !make_packed_map(&maps.a, a_packed, M, K, p.bt))
     return APEX_ERR_CUDA;
-  return launch_gemm<true>(p, tw, ta, a, static_cast<cudaStream_t>(stream));
+  return launch_gemm<true>(p, maps, a, false, static_cast<cudaStream_t>(stream));
 }
 
 apex_status_t apex_get_device_status(void* stream) {
@@ -298,6 +341,12 @@ apex_status_t apex_get_device_status(void* stream) {
 void apex_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns ? ns : 1; }
 
 void apex_debug_withhold_step(int32_t step) { t_withhold = step; }
+
+void apex_debug_trace_next_gemm(uint64_t* trace, int32_t ctas, int32_t steps) {
+  t_trace = reinterpret_cast<unsigned long long*>(trace);
+  t_trace_ctas = ctas;
+  t_trace_steps = steps;
+}
 
 const char* apex_status_string(apex_status_t status) {
   switch (status) {

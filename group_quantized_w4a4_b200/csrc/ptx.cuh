@@ -1,9 +1,9 @@
 // ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, TMA, tcgen05 (TMEM + UMMA).
 //
-// Every wait is bounded: it gives up after a time limit (read from %globaltimer), or when
-// another role of the same CTA has already given up (a shared abort word).  On giving up
-// it records APEX_DEV_TIMEOUT in the library's device status word, so the host can report
-// a timeout instead of the GPU hanging.
+// Every wait is bounded: it gives up after a time limit (counted in SM clock cycles), or
+// when another role of the same CTA has already given up (a shared abort word).  On giving
+// up it records a timeout in the library's device status word, so the host can report it
+// instead of the GPU hanging.
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -57,21 +57,44 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended in hardware for up to `hint_ns` while
+// the phase is incomplete (it resumes as soon as the phase completes), so a waiting warp
+// does not take issue slots from the warps doing work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t clock_cycles() {
+  uint64_t c;
+  asm volatile("mov.u64 %0, %%clock64;" : "=l"(c));
+  return c;
+}
+
 // Wait until the phase with the given parity has completed.  Returns false (and records a
-// timeout) when `limit_ns` elapses first, or when *abort_flag becomes non-zero.
+// timeout) when about `limit_ns` elapses first (measured in SM cycles at 2 cycles per ns,
+// i.e. at most the limit at clocks up to 2 GHz), or when *abort_flag becomes non-zero.
+// Each unsuccessful attempt sleeps in hardware for at most 1 ms (or until the phase
+// completes), so the limit and the abort word are checked at least every millisecond.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
                                           volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const uint64_t t0 = clock_cycles();
   for (uint32_t spin = 1;; ++spin) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((spin & 31u) == 0u) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > limit_ns || spin > (1u << 30)) {
-        atomicOr(&g_device_status, DEV_TIMEOUT);
-        *abort_flag = 1;
-        return false;
-      }
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    if (*abort_flag) return false;
+    if (clock_cycles() - t0 > 2 * limit_ns || spin > (1u << 30)) {
+      atomicOr(&g_device_status, DEV_TIMEOUT);
+      *abort_flag = 1;
+      return false;
     }
   }
 }

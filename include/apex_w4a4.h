@@ -110,11 +110,22 @@ void apex_set_wait_limit_ns(uint64_t ns);
 const char *apex_status_string(apex_status_t status);
 
 /*
- * Test hook: the next GEMM launch on this host thread skips the bulk copy of K-group step
- * `step` (counted within each CTA), so its consumers wait until the time limit.  -1 turns
- * it off.  Used only to test the timeout path; never needed by callers.
+ * Test hook: the next GEMM launch on this host thread skips the bulk copy of pipeline stage
+ * `step` (a pair of K-groups, counted within each CTA), so its consumers wait until the
+ * time limit.  -1 turns it off.  Used only to test the timeout path; never needed by callers.
  */
 void apex_debug_withhold_step(int32_t step);
+
+/*
+ * Tracing hook: the next apex_w4a4_gemm launch on this host thread writes timestamps for
+ * its first `ctas` CTAs (linear block id) into the device buffer trace[ctas][6][steps]
+ * (uint64).  SM clock cycles (clock64): [c][0][s] producer issued stage s (a pair of
+ * K-groups), [c][1][s] converters done with stage s, [c][2][i] MMAs of K-group i issued,
+ * [c][3][i] epilogue done with K-group i, [c][4][i] scales of K-group i loaded;
+ * [c][5][0] / [c][5][1] %globaltimer (ns) at CTA start / end, [c][5][2] the SM it ran on,
+ * [c][5][3] clock64 at CTA start.  Steps beyond `steps` are not recorded.
+ */
+void apex_debug_trace_next_gemm(uint64_t *trace, int32_t ctas, int32_t steps);
 
 #ifdef __cplusplus
 }
