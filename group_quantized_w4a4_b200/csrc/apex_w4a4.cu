@@ -92,21 +92,6 @@ bool make_packed_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K
   return r == CUDA_SUCCESS;
 }
 
-// 2-D map over an fp16 scale matrix [rows][cols]; box = 8 columns (16 bytes) x box_rows.
-// Needs a 16-byte aligned base and cols % 8 == 0 (row stride a multiple of 16 bytes).
-bool make_scale_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
-  cuuint32_t box[2] = {8u, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 // ------------------------------------------------------------------ GEMM planning
 
 struct Plan {
@@ -161,34 +146,28 @@ apex_status_t check_gemm_args(int64_t M, int64_t N, int64_t K, int32_t ga, int32
 }
 
 struct Maps {
-  CUtensorMap w, a, sa, sw;
+  CUtensorMap w, a;
 };
 
-template <int BT, bool DUMP, bool SCT>
+template <int BT, bool DUMP>
 apex_status_t launch_bt(const Plan& p, const Maps& m, const GemmArgs& a, cudaStream_t s) {
   using C = GemmCfg<BT>;
-  auto kern = apex::w4a4_gemm_kernel<BT, DUMP, SCT>;
+  auto kern = apex::w4a4_gemm_kernel<BT, DUMP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return APEX_ERR_CUDA;
   dim3 grid(p.tiles_n, p.tiles_m, a.splits);
-  kern<<<grid, C::THREADS, C::SMEM, s>>>(m.w, m.a, m.sa, m.sw, a);
+  kern<<<grid, C::THREADS, C::SMEM, s>>>(m.w, m.a, a);
   return cuda_status(cudaPeekAtLastError());
 }
 
-template <bool DUMP, bool SCT>
-apex_status_t launch_gemm_sct(const Plan& p, const Maps& m, const GemmArgs& a, cudaStream_t s) {
-  switch (p.bt) {
-    case 16: return launch_bt<16, DUMP, SCT>(p, m, a, s);
-    case 32: return launch_bt<32, DUMP, SCT>(p, m, a, s);
-    case 64: return launch_bt<64, DUMP, SCT>(p, m, a, s);
-    default: return launch_bt<128, DUMP, SCT>(p, m, a, s);
-  }
-}
-
 template <bool DUMP>
-apex_status_t launch_gemm(const Plan& p, const Maps& m, const GemmArgs& a, bool sct,
-                          cudaStream_t s) {
-  return sct ? launch_gemm_sct<DUMP, true>(p, m, a, s) : launch_gemm_sct<DUMP, false>(p, m, a, s);
+apex_status_t launch_gemm(const Plan& p, const Maps& m, const GemmArgs& a, cudaStream_t s) {
+  switch (p.bt) {
+    case 16: return launch_bt<16, DUMP>(p, m, a, s);
+    case 32: return launch_bt<32, DUMP>(p, m, a, s);
+    case 64: return launch_bt<64, DUMP>(p, m, a, s);
+    default: return launch_bt<128, DUMP>(p, m, a, s);
+  }
 }
 
 apex_status_t quantize_launch(const void* x, int64_t rows, int64_t K, int32_t group, void* packed,
@@ -254,9 +233,10 @@ apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, i
   while (p.splits > 1 && (!workspace || workspace_for(p, M, N) > workspace_bytes)) --p.splits;
   const int G = (int)(K / 128);
   const int Gw = (int)(K / group_w);
-  // Scales by TMA need 16-byte row strides and bases, and splits starting on 8-group blocks.
-  const bool sct = G % 8 == 0 && (Gw % 8 == 0 || Gw == 1) && aligned(a_scales, 16) &&
-                   aligned(w_scales, 16);
+  // Scales are fetched in 16-byte blocks of 8 groups when rows are 16-byte strided and the
+  // splits start on multiples of 8 groups.
+  const bool sa_vec = G % 8 == 0 && aligned(a_scales, 16);
+  const bool sw_vec = group_w == 128 && G % 8 == 0 && aligned(w_scales, 16);
   GemmArgs a{};
   a.M = (int)M;
   a.N = (int)N;
@@ -265,7 +245,9 @@ apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, i
   a.G = G;
   a.Gw = Gw;
   a.gps = (G + p.splits - 1) / p.splits;
-  if (sct) a.gps = (a.gps + 7) / 8 * 8;
+  if (sa_vec || sw_vec) a.gps = (a.gps + 7) / 8 * 8;
+  a.sa_vec = sa_vec;
+  a.sw_vec = sw_vec;
   a.splits = (G + a.gps - 1) / a.gps;  // no empty split
   p.splits = a.splits;
   a.sa = static_cast<const __half*>(a_scales);
@@ -289,11 +271,7 @@ apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, i
   if (!make_packed_map(&maps.w, w_packed, N, K, 128) ||
       !make_packed_map(&maps.a, a_packed, M, K, p.bt))
     return APEX_ERR_CUDA;
-  if (sct) {
-    if (!make_scale_map(&maps.sa, a_scales, M, G, p.bt)) return APEX_ERR_CUDA;
-    if (Gw % 8 == 0 && !make_scale_map(&maps.sw, w_scales, N, Gw, 128)) return APEX_ERR_CUDA;
-  }
-  return launch_gemm<false>(p, maps, a, sct, static_cast<cudaStream_t>(stream));
+  return launch_gemm<false>(p, maps, a, static_cast<cudaStream_t>(stream));
 }
 
 apex_status_t apex_w4a4_group_partials(int64_t M, int64_t N, int64_t K, const void* a_packed,
@@ -323,7 +301,7 @@ apex_status_t apex_w4a4_group_partials(int64_t M, int64_t N, int64_t K, const vo
   if (!make_packed_map(&maps.w, w_packed, N, K, 128) ||
       !make_packed_map(&maps.a, a_packed, M, K, p.bt))
     return APEX_ERR_CUDA;
-  return launch_gemm<true>(p, maps, a, false, static_cast<cudaStream_t>(stream));
+  return launch_gemm<true>(p, maps, a, static_cast<cudaStream_t>(stream));
 }
 
 apex_status_t apex_get_device_status(void* stream) {
