@@ -21,6 +21,7 @@ import threading
 __all__ = [
     "ApexError", "load_library", "library_path",
     "apex_pack_weights_int4", "apex_quantize_act_int4", "apex_w4a4_gemm",
+    "apex_w4a4_gemm_noalloc",
     "apex_w4a4_gemm_workspace_size", "apex_w4a4_group_partials", "apex_get_device_status",
     "apex_set_wait_limit_ns", "apex_status_string", "apex_debug_withhold_step",
     "apex_debug_trace_next_gemm",
@@ -71,6 +72,8 @@ def load_library(build_if_missing: bool = True):
         lib.apex_quantize_act_int4.restype = st
         lib.apex_w4a4_gemm.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P, SZ, P]
         lib.apex_w4a4_gemm.restype = st
+        lib.apex_w4a4_gemm_noalloc.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P]
+        lib.apex_w4a4_gemm_noalloc.restype = st
         lib.apex_w4a4_gemm_workspace_size.argtypes = [I64, I64, I64, I32, I32]
         lib.apex_w4a4_gemm_workspace_size.restype = SZ
         lib.apex_w4a4_group_partials.argtypes = [I64, I64, I64, P, P, P, P]
@@ -143,6 +146,16 @@ def apex_w4a4_gemm(M, N, K, group_a, group_w, a_packed, a_scales, w_packed, w_sc
                                          _ptr(y_f16), _ptr(workspace), workspace_bytes or 0,
                                          _stream(stream)),
            "apex_w4a4_gemm")
+
+
+def apex_w4a4_gemm_noalloc(M, N, K, group_a, group_w, a_packed, a_scales, w_packed, w_scales,
+                           y_f16, stream=None):
+    """apex_w4a4_gemm without a workspace argument: for callers that may not allocate device
+    memory at call time; the split-K scratch is a fixed array inside the library."""
+    _check(load_library().apex_w4a4_gemm_noalloc(M, N, K, group_a, group_w, _ptr(a_packed),
+                                                 _ptr(a_scales), _ptr(w_packed),
+                                                 _ptr(w_scales), _ptr(y_f16), _stream(stream)),
+           "apex_w4a4_gemm_noalloc")
 
 
 def apex_w4a4_gemm_workspace_size(M, N, K, group_a, group_w) -> int:

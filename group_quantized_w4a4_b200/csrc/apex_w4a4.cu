@@ -274,6 +274,92 @@ apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, i
   return launch_gemm<false>(p, maps, a, static_cast<cudaStream_t>(stream));
 }
 
+// ------------------------------------------------------------------ allocation-free GEMM
+//
+// For callers that may not allocate device memory while they run: serving runtimes that
+// plan every device byte ahead of time and hand out no scratch, plugin hosts whose
+// allocator is off limits to the plugin, and code paths that must not pay for
+// cudaMalloc/cudaFree (which can stall or synchronize the whole device).  The split-K
+// scratch lives in this fixed, library-owned device array instead: every GPU that loads
+// the library keeps APEX_STATIC_SCRATCH_BYTES reserved until the process exits.
+static __device__ __align__(256) uint8_t g_static_scratch[APEX_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of g_static_scratch, looked up once per device (with that device current)
+// on the first call there.  The array's host-side name is only a handle, never an address.
+apex_status_t static_scratch_ptr(void** out) {
+  static std::mutex mu;
+  static void* ptrs[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return APEX_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return APEX_ERR_CUDA;
+    ptrs[dev] = p;
+  }
+  *out = ptrs[dev];
+  return APEX_OK;
+}
+
+}  // namespace
+
+apex_status_t apex_w4a4_gemm_noalloc(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                     int32_t group_w, const void* a_packed, const void* a_scales,
+                                     const void* w_packed, const void* w_scales, void* y_f16,
+                                     void* stream) {
+  apex_status_t st = check_gemm_args(M, N, K, group_a, group_w);
+  if (st != APEX_OK) return st;
+  if (!a_packed || !a_scales || !w_packed || !w_scales || !y_f16) return APEX_ERR_INVALID_ARG;
+  if (!aligned(a_packed, 16) || !aligned(w_packed, 16) || !aligned(a_scales, 2) ||
+      !aligned(w_scales, 2) || !aligned(y_f16, 2))
+    return APEX_ERR_ALIGNMENT;
+
+  Plan p = make_plan(M, N, K);
+  const int G = (int)(K / 128);
+  const int Gw = (int)(K / group_w);
+  const bool sa_vec = G % 8 == 0 && aligned(a_scales, 16);
+  const bool sw_vec = group_w == 128 && G % 8 == 0 && aligned(w_scales, 16);
+  GemmArgs a{};
+  a.M = (int)M;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.gw = group_w;
+  a.G = G;
+  a.Gw = Gw;
+  a.gps = (G + p.splits - 1) / p.splits;
+  if (sa_vec || sw_vec) a.gps = (a.gps + 7) / 8 * 8;
+  a.sa_vec = sa_vec;
+  a.sw_vec = sw_vec;
+  a.splits = (G + a.gps - 1) / a.gps;
+  p.splits = a.splits;
+  // The problem's split-K scratch must fit the fixed array; larger problems are refused.
+  if (workspace_for(p, M, N) > (size_t)APEX_STATIC_SCRATCH_BYTES) return APEX_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (p.splits > 1) {
+    void* scratch = nullptr;
+    st = static_scratch_ptr(&scratch);
+    if (st != APEX_OK) return st;
+    // The array keeps whatever the previous call left: the arrival counters start at zero.
+    if (cudaMemsetAsync(scratch, 0, counters_bytes(p), s) != cudaSuccess) return APEX_ERR_CUDA;
+    a.counters = static_cast<unsigned*>(scratch);
+    a.ws = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + counters_bytes(p));
+  }
+  a.sa = static_cast<const __half*>(a_scales);
+  a.sw = static_cast<const __half*>(w_scales);
+  a.y = static_cast<__half*>(y_f16);
+  a.dump = nullptr;
+  a.wait_ns = g_wait_limit_ns;
+  a.withhold = -1;
+  Maps maps;
+  memset(&maps, 0, sizeof(maps));
+  if (!make_packed_map(&maps.w, w_packed, N, K, 128) ||
+      !make_packed_map(&maps.a, a_packed, M, K, p.bt))
+    return APEX_ERR_CUDA;
+  return launch_gemm<false>(p, maps, a, s);
+}
+
 apex_status_t apex_w4a4_group_partials(int64_t M, int64_t N, int64_t K, const void* a_packed,
                                        const void* w_packed, int32_t* partials_i32,
                                        void* stream) {

@@ -81,6 +81,29 @@ apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, i
                              const void *w_scales, void *y_f16, void *workspace,
                              size_t workspace_bytes, void *stream);
 
+/*
+ * Allocation-free variant of apex_w4a4_gemm.  The paper has no counterpart: this entry
+ * point exists for callers that cannot allocate device memory while they run -- serving
+ * runtimes that budget every device byte up front and hand out no scratch, plugin hosts
+ * whose allocator the plugin may not call, and latency-critical paths that must avoid
+ * cudaMalloc/cudaFree because those can stall or synchronize the device.
+ * It computes exactly what apex_w4a4_gemm computes, with the same operand rules, but takes
+ * no workspace: its split-K scratch is a fixed array of APEX_STATIC_SCRATCH_BYTES inside
+ * the library, reserved on every GPU that loads the library until the process exits.  It
+ * calls no allocator.  A problem whose scratch would exceed that size is refused with
+ * APEX_ERR_UNSUPPORTED.
+ * The first call on each device looks the array's device address up (with that device
+ * current), so make that first call before any stream capture.  All calls on a device
+ * share the one array and it keeps the previous call's contents (each call clears the
+ * parts that must start at zero), so calls that overlap on the GPU -- on different
+ * streams, or from different host threads -- race and must be ordered by the caller.
+ */
+#define APEX_STATIC_SCRATCH_BYTES (8u << 20)
+apex_status_t apex_w4a4_gemm_noalloc(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                     int32_t group_w, const void *a_packed, const void *a_scales,
+                                     const void *w_packed, const void *w_scales, void *y_f16,
+                                     void *stream);
+
 /* Workspace bytes apex_w4a4_gemm would use for this problem (0 when it needs none). */
 size_t apex_w4a4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group_a,
                                      int32_t group_w);
