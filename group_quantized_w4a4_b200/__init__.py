@@ -21,7 +21,8 @@ import threading
 __all__ = [
     "ApexError", "load_library", "library_path",
     "apex_pack_weights_int4", "apex_quantize_act_int4", "apex_w4a4_gemm",
-    "apex_w4a4_gemm_noalloc",
+    "apex_w4a4_gemm_noalloc", "apex_quantize_act_int4_expanded", "apex_w4a4_gemm_expanded",
+    "quantize_act_expanded",
     "apex_w4a4_gemm_workspace_size", "apex_w4a4_group_partials", "apex_get_device_status",
     "apex_set_wait_limit_ns", "apex_status_string", "apex_debug_withhold_step",
     "apex_debug_trace_next_gemm",
@@ -70,6 +71,10 @@ def load_library(build_if_missing: bool = True):
         lib.apex_pack_weights_int4.restype = st
         lib.apex_quantize_act_int4.argtypes = [P, I64, I64, I32, P, P, P]
         lib.apex_quantize_act_int4.restype = st
+        lib.apex_quantize_act_int4_expanded.argtypes = [P, I64, I64, I32, P, P, P]
+        lib.apex_quantize_act_int4_expanded.restype = st
+        lib.apex_w4a4_gemm_expanded.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P, SZ, P]
+        lib.apex_w4a4_gemm_expanded.restype = st
         lib.apex_w4a4_gemm.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P, SZ, P]
         lib.apex_w4a4_gemm.restype = st
         lib.apex_w4a4_gemm_noalloc.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P]
@@ -148,6 +153,34 @@ def apex_w4a4_gemm(M, N, K, group_a, group_w, a_packed, a_scales, w_packed, w_sc
            "apex_w4a4_gemm")
 
 
+def apex_quantize_act_int4_expanded(x_f16, M, K, group_a, x_q8, x_scales_f16, stream=None):
+    _check(load_library().apex_quantize_act_int4_expanded(_ptr(x_f16), M, K, group_a,
+                                                          _ptr(x_q8), _ptr(x_scales_f16),
+                                                          _stream(stream)),
+           "apex_quantize_act_int4_expanded")
+
+
+def apex_w4a4_gemm_expanded(M, N, K, group_a, group_w, a_q8, a_scales, w_packed, w_scales,
+                            y_f16, workspace=None, workspace_bytes=None, stream=None):
+    if workspace is not None and workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(load_library().apex_w4a4_gemm_expanded(M, N, K, group_a, group_w, _ptr(a_q8),
+                                                  _ptr(a_scales), _ptr(w_packed),
+                                                  _ptr(w_scales), _ptr(y_f16), _ptr(workspace),
+                                                  workspace_bytes or 0, _stream(stream)),
+           "apex_w4a4_gemm_expanded")
+
+
+def quantize_act_expanded(x, group_a: int = 128, stream=None):
+    """fp16 [M, K] CUDA tensor -> (expanded int8 [M, K], scales fp16 [M, K/group_a])."""
+    import torch
+    M, K = x.shape
+    q8 = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((M, K // group_a), dtype=torch.float16, device=x.device)
+    apex_quantize_act_int4_expanded(x, M, K, group_a, q8, scales, stream)
+    return q8, scales
+
+
 def apex_w4a4_gemm_noalloc(M, N, K, group_a, group_w, a_packed, a_scales, w_packed, w_scales,
                            y_f16, stream=None):
     """apex_w4a4_gemm without a workspace argument: for callers that may not allocate device
@@ -181,8 +214,8 @@ def apex_debug_withhold_step(step: int):
 
 
 def apex_debug_trace_next_gemm(trace, ctas: int, steps: int):
-    """trace: int64 CUDA tensor with at least ctas*6*steps elements (zeroed by the caller)."""
-    if trace.numel() < ctas * 6 * steps:
+    """trace: int64 CUDA tensor with at least ctas*10*steps elements (zeroed by the caller)."""
+    if trace.numel() < ctas * 10 * steps:
         raise ValueError("trace buffer too small")
     load_library().apex_debug_trace_next_gemm(_ptr(trace), int(ctas), int(steps))
 

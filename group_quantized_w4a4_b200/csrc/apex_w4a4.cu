@@ -92,12 +92,30 @@ bool make_packed_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K
   return r == CUDA_SUCCESS;
 }
 
+// 2-D map over expanded activations [rows][K] bytes (16*q per element); box = 128 bytes
+// (one 128-wide K-group) x box_rows rows, 128-byte swizzle: it lands in shared memory in the
+// tensor core's K-major operand layout.
+bool make_expanded_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K};
+  cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ GEMM planning
 
 struct Plan {
   int bt = 128;
-  int splits = 1;
-  int tiles_n = 0, tiles_m = 0;
+  int tiles_n = 0, tiles_m = 0, T = 0;
+  int S = 0;        // K-stages (pairs of groups) per tile
+  int P = 0;        // persistent CTAs
+  int streamk = 0;  // stream-K partition (needs workspace) or whole tiles round-robin
 };
 
 int pick_bt(int64_t M) {
@@ -107,32 +125,33 @@ int pick_bt(int64_t M) {
   return 128;
 }
 
-int ctas_per_sm(int bt) { return bt <= 32 ? 2 : 1; }
-
-Plan make_plan(int64_t M, int64_t N, int64_t K) {
+// One persistent CTA per SM.  Whole tiles when there are at least 4 per SM (the last,
+// partial round costs little); otherwise stream-K, so every SM streams the same bytes.
+Plan make_plan(int64_t M, int64_t N, int64_t K, bool allow_streamk) {
   Plan p;
   p.bt = pick_bt(M);
   p.tiles_n = (int)((N + 127) / 128);
   p.tiles_m = (int)((M + p.bt - 1) / p.bt);
-  const int64_t tiles = (int64_t)p.tiles_n * p.tiles_m;
+  p.T = p.tiles_n * p.tiles_m;
   const int G = (int)(K / 128);
-  const int64_t slots = (int64_t)dev_info().sms * ctas_per_sm(p.bt);
-  if (tiles < slots) {
-    int s = (int)(slots / tiles);
-    const int min_groups = 4;
-    s = s < G / min_groups ? s : G / min_groups;
-    p.splits = s > 1 ? s : 1;
+  p.S = (G + 1) / 2;
+  const int sms = dev_info().sms;
+  if (!allow_streamk || p.T >= 4 * sms) {
+    p.streamk = 0;
+    p.P = p.T < sms ? p.T : sms;
+  } else {
+    p.streamk = 1;
+    const long long units = (long long)p.T * p.S;
+    p.P = units < sms ? (int)units : sms;
   }
   return p;
 }
 
-size_t counters_bytes(const Plan& p) {
-  return (((size_t)p.tiles_n * p.tiles_m * 4) + 255) & ~(size_t)255;
-}
+size_t counters_bytes(const Plan& p) { return (((size_t)p.T * 4) + 255) & ~(size_t)255; }
 
-size_t workspace_for(const Plan& p, int64_t M, int64_t N) {
-  if (p.splits <= 1) return 0;
-  return counters_bytes(p) + (size_t)p.splits * (size_t)M * (size_t)N * 4;
+size_t workspace_for(const Plan& p) {
+  if (!p.streamk) return 0;
+  return counters_bytes(p) + (size_t)p.P * 2 * (size_t)p.bt * 128 * 4;
 }
 
 apex_status_t check_gemm_args(int64_t M, int64_t N, int64_t K, int32_t ga, int32_t gw) {
@@ -149,32 +168,65 @@ struct Maps {
   CUtensorMap w, a;
 };
 
-template <int BT, bool DUMP>
+template <int BT, int MODE>
 apex_status_t launch_bt(const Plan& p, const Maps& m, const GemmArgs& a, cudaStream_t s) {
-  using C = GemmCfg<BT>;
-  auto kern = apex::w4a4_gemm_kernel<BT, DUMP>;
+  using C = GemmCfg<BT, MODE>;
+  auto kern = apex::w4a4_gemm_kernel<BT, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return APEX_ERR_CUDA;
-  dim3 grid(p.tiles_n, p.tiles_m, a.splits);
-  kern<<<grid, C::THREADS, C::SMEM, s>>>(m.w, m.a, a);
+  kern<<<p.P, C::THREADS, C::SMEM, s>>>(m.w, m.a, a);
   return cuda_status(cudaPeekAtLastError());
 }
 
-template <bool DUMP>
+template <int MODE>
 apex_status_t launch_gemm(const Plan& p, const Maps& m, const GemmArgs& a, cudaStream_t s) {
   switch (p.bt) {
-    case 16: return launch_bt<16, DUMP>(p, m, a, s);
-    case 32: return launch_bt<32, DUMP>(p, m, a, s);
-    case 64: return launch_bt<64, DUMP>(p, m, a, s);
-    default: return launch_bt<128, DUMP>(p, m, a, s);
+    case 16: return launch_bt<16, MODE>(p, m, a, s);
+    case 32: return launch_bt<32, MODE>(p, m, a, s);
+    case 64: return launch_bt<64, MODE>(p, m, a, s);
+    default: return launch_bt<128, MODE>(p, m, a, s);
   }
 }
 
+// Fills the fields every mode shares.
+GemmArgs base_args(const Plan& p, int64_t M, int64_t N, int64_t K, int32_t gw,
+                   const void* a_scales, const void* w_scales, void* y) {
+  GemmArgs a{};
+  a.M = (int)M;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.gw = gw;
+  a.G = (int)(K / 128);
+  a.Gw = (int)(K / gw);
+  a.tiles_n = p.tiles_n;
+  a.tiles_m = p.tiles_m;
+  a.T = p.T;
+  a.S = p.S;
+  a.P = p.P;
+  a.streamk = p.streamk;
+  // Scales are fetched in 16-byte blocks of 8 groups when rows are 16-byte strided.
+  a.sa_vec = a.G % 8 == 0 && a_scales && aligned(a_scales, 16);
+  a.sw_vec = gw == 128 && a.G % 8 == 0 && w_scales && aligned(w_scales, 16);
+  a.sa = static_cast<const __half*>(a_scales);
+  a.sw = static_cast<const __half*>(w_scales);
+  a.y = static_cast<__half*>(y);
+  a.wait_ns = g_wait_limit_ns;
+  a.withhold = -1;
+  return a;
+}
+
+void attach_workspace(const Plan& p, GemmArgs& a, void* ws) {
+  if (!p.streamk) return;
+  a.counters = static_cast<unsigned*>(ws);
+  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + counters_bytes(p));
+}
+
 apex_status_t quantize_launch(const void* x, int64_t rows, int64_t K, int32_t group, void* packed,
-                              void* scales, void* stream) {
+                              void* scales, void* stream, bool expanded = false) {
   if (!x || !packed || !scales) return APEX_ERR_INVALID_ARG;
   if (rows <= 0 || K <= 0 || group <= 0 || K % group || group % 128) return APEX_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(packed, 4) || !aligned(scales, 2)) return APEX_ERR_ALIGNMENT;
+  if (!aligned(x, 16) || !aligned(packed, expanded ? 8 : 4) || !aligned(scales, 2))
+    return APEX_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t units = rows * (K / group);
   const int threads = 256;
@@ -186,7 +238,11 @@ apex_status_t quantize_launch(const void* x, int64_t rows, int64_t K, int32_t gr
   const __half* xh = static_cast<const __half*>(x);
   uint8_t* pk = static_cast<uint8_t*>(packed);
   __half* sc = static_cast<__half*>(scales);
-  if (group == 128)
+  if (expanded) {
+    if (group != 128) return APEX_ERR_UNSUPPORTED;
+    apex::quantize_pack_kernel<1, true><<<(unsigned)blocks, threads, 0, s>>>(xh, rows, K, group, pk,
+                                                                             sc);
+  } else if (group == 128)
     apex::quantize_pack_kernel<1><<<(unsigned)blocks, threads, 0, s>>>(xh, rows, K, group, pk, sc);
   else if (group == 256)
     apex::quantize_pack_kernel<2><<<(unsigned)blocks, threads, 0, s>>>(xh, rows, K, group, pk, sc);
@@ -211,10 +267,42 @@ apex_status_t apex_quantize_act_int4(const void* x_f16, int64_t M, int64_t K, in
   return quantize_launch(x_f16, M, K, group_a, x_packed_u8, x_scales_f16, stream);
 }
 
+apex_status_t apex_quantize_act_int4_expanded(const void* x_f16, int64_t M, int64_t K,
+                                              int32_t group_a, void* x_q8, void* x_scales_f16,
+                                              void* stream) {
+  return quantize_launch(x_f16, M, K, group_a, x_q8, x_scales_f16, stream, true);
+}
+
+apex_status_t apex_w4a4_gemm_expanded(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                      int32_t group_w, const void* a_q8, const void* a_scales,
+                                      const void* w_packed, const void* w_scales, void* y_f16,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+  apex_status_t st = check_gemm_args(M, N, K, group_a, group_w);
+  if (st != APEX_OK) return st;
+  if (!a_q8 || !a_scales || !w_packed || !w_scales || !y_f16) return APEX_ERR_INVALID_ARG;
+  if (!aligned(a_q8, 16) || !aligned(w_packed, 16) || !aligned(a_scales, 2) ||
+      !aligned(w_scales, 2) || !aligned(y_f16, 2) || (workspace && !aligned(workspace, 256)))
+    return APEX_ERR_ALIGNMENT;
+  Plan p = make_plan(M, N, K, true);
+  if (p.streamk && (!workspace || workspace_for(p) > workspace_bytes)) p = make_plan(M, N, K, false);
+  GemmArgs a = base_args(p, M, N, K, group_w, a_scales, w_scales, y_f16);
+  attach_workspace(p, a, workspace);
+  a.trace = t_trace;
+  a.trace_ctas = t_trace_ctas;
+  a.trace_steps = t_trace_steps;
+  t_trace = nullptr;
+  Maps maps;
+  memset(&maps, 0, sizeof(maps));
+  if (!make_packed_map(&maps.w, w_packed, N, K, 128) ||
+      !make_expanded_map(&maps.a, a_q8, M, K, p.bt))
+    return APEX_ERR_CUDA;
+  return launch_gemm<apex::MODE_AQ8>(p, maps, a, static_cast<cudaStream_t>(stream));
+}
+
 size_t apex_w4a4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group_a,
                                      int32_t group_w) {
   if (check_gemm_args(M, N, K, group_a, group_w) != APEX_OK) return 0;
-  return workspace_for(make_plan(M, N, K), M, N);
+  return workspace_for(make_plan(M, N, K, true));
 }
 
 apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, int32_t group_w,
@@ -228,37 +316,11 @@ apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, i
       !aligned(w_scales, 2) || !aligned(y_f16, 2) || (workspace && !aligned(workspace, 256)))
     return APEX_ERR_ALIGNMENT;
 
-  Plan p = make_plan(M, N, K);
-  // Shrink the split to what the caller's workspace holds.
-  while (p.splits > 1 && (!workspace || workspace_for(p, M, N) > workspace_bytes)) --p.splits;
-  const int G = (int)(K / 128);
-  const int Gw = (int)(K / group_w);
-  // Scales are fetched in 16-byte blocks of 8 groups when rows are 16-byte strided and the
-  // splits start on multiples of 8 groups.
-  const bool sa_vec = G % 8 == 0 && aligned(a_scales, 16);
-  const bool sw_vec = group_w == 128 && G % 8 == 0 && aligned(w_scales, 16);
-  GemmArgs a{};
-  a.M = (int)M;
-  a.N = (int)N;
-  a.K = (int)K;
-  a.gw = group_w;
-  a.G = G;
-  a.Gw = Gw;
-  a.gps = (G + p.splits - 1) / p.splits;
-  if (sa_vec || sw_vec) a.gps = (a.gps + 7) / 8 * 8;
-  a.sa_vec = sa_vec;
-  a.sw_vec = sw_vec;
-  a.splits = (G + a.gps - 1) / a.gps;  // no empty split
-  p.splits = a.splits;
-  a.sa = static_cast<const __half*>(a_scales);
-  a.sw = static_cast<const __half*>(w_scales);
-  a.y = static_cast<__half*>(y_f16);
-  if (p.splits > 1) {
-    a.counters = static_cast<unsigned*>(workspace);
-    a.ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + counters_bytes(p));
-  }
-  a.dump = nullptr;
-  a.wait_ns = g_wait_limit_ns;
+  Plan p = make_plan(M, N, K, true);
+  // Without a large enough workspace, whole tiles only.
+  if (p.streamk && (!workspace || workspace_for(p) > workspace_bytes)) p = make_plan(M, N, K, false);
+  GemmArgs a = base_args(p, M, N, K, group_w, a_scales, w_scales, y_f16);
+  attach_workspace(p, a, workspace);
   a.withhold = t_withhold;
   t_withhold = -1;
   a.trace = t_trace;
@@ -271,7 +333,7 @@ apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, i
   if (!make_packed_map(&maps.w, w_packed, N, K, 128) ||
       !make_packed_map(&maps.a, a_packed, M, K, p.bt))
     return APEX_ERR_CUDA;
-  return launch_gemm<false>(p, maps, a, static_cast<cudaStream_t>(stream));
+  return launch_gemm<apex::MODE_PACKED>(p, maps, a, static_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------------------ allocation-free GEMM
@@ -316,48 +378,25 @@ apex_status_t apex_w4a4_gemm_noalloc(int64_t M, int64_t N, int64_t K, int32_t gr
       !aligned(w_scales, 2) || !aligned(y_f16, 2))
     return APEX_ERR_ALIGNMENT;
 
-  Plan p = make_plan(M, N, K);
-  const int G = (int)(K / 128);
-  const int Gw = (int)(K / group_w);
-  const bool sa_vec = G % 8 == 0 && aligned(a_scales, 16);
-  const bool sw_vec = group_w == 128 && G % 8 == 0 && aligned(w_scales, 16);
-  GemmArgs a{};
-  a.M = (int)M;
-  a.N = (int)N;
-  a.K = (int)K;
-  a.gw = group_w;
-  a.G = G;
-  a.Gw = Gw;
-  a.gps = (G + p.splits - 1) / p.splits;
-  if (sa_vec || sw_vec) a.gps = (a.gps + 7) / 8 * 8;
-  a.sa_vec = sa_vec;
-  a.sw_vec = sw_vec;
-  a.splits = (G + a.gps - 1) / a.gps;
-  p.splits = a.splits;
-  // The problem's split-K scratch must fit the fixed array; larger problems are refused.
-  if (workspace_for(p, M, N) > (size_t)APEX_STATIC_SCRATCH_BYTES) return APEX_ERR_UNSUPPORTED;
+  Plan p = make_plan(M, N, K, true);
+  // The problem's stream-K scratch must fit the fixed array; larger problems are refused.
+  if (workspace_for(p) > (size_t)APEX_STATIC_SCRATCH_BYTES) return APEX_ERR_UNSUPPORTED;
+  GemmArgs a = base_args(p, M, N, K, group_w, a_scales, w_scales, y_f16);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (p.splits > 1) {
+  if (p.streamk) {
     void* scratch = nullptr;
     st = static_scratch_ptr(&scratch);
     if (st != APEX_OK) return st;
     // The array keeps whatever the previous call left: the arrival counters start at zero.
     if (cudaMemsetAsync(scratch, 0, counters_bytes(p), s) != cudaSuccess) return APEX_ERR_CUDA;
-    a.counters = static_cast<unsigned*>(scratch);
-    a.ws = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + counters_bytes(p));
+    attach_workspace(p, a, scratch);
   }
-  a.sa = static_cast<const __half*>(a_scales);
-  a.sw = static_cast<const __half*>(w_scales);
-  a.y = static_cast<__half*>(y_f16);
-  a.dump = nullptr;
-  a.wait_ns = g_wait_limit_ns;
-  a.withhold = -1;
   Maps maps;
   memset(&maps, 0, sizeof(maps));
   if (!make_packed_map(&maps.w, w_packed, N, K, 128) ||
       !make_packed_map(&maps.a, a_packed, M, K, p.bt))
     return APEX_ERR_CUDA;
-  return launch_gemm<false>(p, maps, a, s);
+  return launch_gemm<apex::MODE_PACKED>(p, maps, a, s);
 }
 
 apex_status_t apex_w4a4_group_partials(int64_t M, int64_t N, int64_t K, const void* a_packed,
@@ -368,26 +407,15 @@ apex_status_t apex_w4a4_group_partials(int64_t M, int64_t N, int64_t K, const vo
   if (!a_packed || !w_packed || !partials_i32) return APEX_ERR_INVALID_ARG;
   if (!aligned(a_packed, 16) || !aligned(w_packed, 16) || !aligned(partials_i32, 4))
     return APEX_ERR_ALIGNMENT;
-  Plan p = make_plan(M, N, K);
-  p.splits = 1;
-  GemmArgs a{};
-  a.M = (int)M;
-  a.N = (int)N;
-  a.K = (int)K;
-  a.gw = 128;
-  a.G = (int)(K / 128);
-  a.Gw = a.G;
-  a.gps = a.G;
-  a.splits = 1;
+  Plan p = make_plan(M, N, K, false);
+  GemmArgs a = base_args(p, M, N, K, 128, nullptr, nullptr, nullptr);
   a.dump = partials_i32;
-  a.wait_ns = g_wait_limit_ns;
-  a.withhold = -1;
   Maps maps;
   memset(&maps, 0, sizeof(maps));
   if (!make_packed_map(&maps.w, w_packed, N, K, 128) ||
       !make_packed_map(&maps.a, a_packed, M, K, p.bt))
     return APEX_ERR_CUDA;
-  return launch_gemm<true>(p, maps, a, static_cast<cudaStream_t>(stream));
+  return launch_gemm<apex::MODE_DUMP>(p, maps, a, static_cast<cudaStream_t>(stream));
 }
 
 apex_status_t apex_get_device_status(void* stream) {

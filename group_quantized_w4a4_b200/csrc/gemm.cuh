@@ -6,32 +6,41 @@
 // INT4 tensor-core products with per-group dequantisation on the CUDA cores; the
 // mixed-granularity mode keeps 128-wide activation groups and coarser weight groups).
 //
-// Tile: 128 weight rows (n) x BT tokens (m) per CTA, one K-group (128) per MMA step.
-// The MMA runs "weight-stationary": the tensor core's A operand (M = 128) is the weight
-// tile held in tensor memory, its B operand (N = BT) the token tile in shared memory, so a
-// 16-token decode still uses the full 128-row MMA.  Roles:
-//   warp 0      TMA producer: packed W tile [128 x 128 B] and packed A tile [BT x 128 B],
-//               two K-groups per stage, into a ring of shared-memory stages (128-byte
-//               swizzle).
+// Tile: 128 weight rows (n) x BT tokens (m), one K-group (128) per MMA step.  The MMA runs
+// "weight-stationary": the tensor core's A operand (M = 128) is the weight tile held in
+// tensor memory, its B operand (N = BT) the token tile in shared memory, so a 16-token
+// decode still uses the full 128-row MMA.
+//
+// Persistent CTAs, one per SM, walk a list of segments (tile, K-group range):
+//   tile mode     whole tiles, round-robin over the CTAs (many tiles);
+//   stream-K      the tiles' K-stages are cut into equal contiguous ranges, one per CTA, so
+//                 every SM streams the same number of bytes (few tiles: decode, small M).
+//                 A tile covered by several CTAs is finished by the last one to arrive,
+//                 which adds the fp32 partials in CTA order (deterministic).
+// Roles:
+//   warp 0      TMA producer: packed W tile [128 x 128 B] (two K-groups per stage) and
+//               the token tile -- packed [BT x 128 B], or, in the expanded-activation mode,
+//               one [BT x 128 B] int8 tile per group straight into the MMA operand slot.
 //   warp 1      MMA issuer (one thread): 4 x tcgen05.mma kind::i8 (K = 32 each) per group
 //               into a tensor-memory slot; one exact int32 partial per group.
-//   warps 2-5   converters: nibbles -> int8 in registers.  The weight row of each thread
-//               goes to tensor memory (tcgen05.st); the token rows go to shared memory in
-//               the 128-byte-swizzled K-major operand layout.
-//   warps 6..   epilogue: tcgen05.ld of a group's partials while the next groups' MMAs
+//   warps 2..   converters (one warpgroup, or two taking alternate stages for narrow
+//               tiles): nibbles -> int8 in registers.  The weight row of each thread goes to
+//               tensor memory (tcgen05.st); packed token rows go to shared memory in the
+//               128-byte-swizzled K-major operand layout.
+//   then        epilogue: tcgen05.ld of a group's partials while the next groups' MMAs
 //               run, fp32 scale by sa*sw and accumulate in registers (packed f32x2 math);
 //               fp16 output.  Each epilogue thread also fetches the scales it needs, one
 //               block of 8 groups ahead (its weight row's sw; one token's sa, shared with
 //               the other epilogue threads through a small transposed buffer).
 // A warp reaches tensor-memory lanes 32*(warp % 4) .. +31 only, so each group of four
-// consecutive warps covers the 128 lanes once (the converter warps 2-5 are lane quarters
-// 2,3,0,1; the epilogue warps 6-9 too).
+// consecutive warps covers the 128 lanes once.
 //
 // Nibble expansion: for a 32-bit word w of 8 packed nibbles, (w << 4) & 0xF0F0F0F0 holds
 // 16*q for the 4 even k and w & 0xF0F0F0F0 16*q for the 4 odd k, as signed bytes.  Both
 // operands get the same within-group K order (even k of a word, then odd k), so each
 // group's sum is unchanged; the tensor core returns 256*P_g exactly (|256 P_g| <= 2^21),
-// and the factor 1/256 is folded into the weight scale.
+// and the factor 1/256 is folded into the weight scale.  The expanded activations written
+// by the quantizer use the same order and values (16*q).
 #pragma once
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -41,26 +50,32 @@
 
 namespace apex {
 
+enum GemmMode : int { MODE_PACKED = 0, MODE_AQ8 = 1, MODE_DUMP = 2 };
+
 struct GemmArgs {
   int M, N, K;
   int gw;            // weight group (multiple of 128 dividing K)
   int G;             // K / 128
   int Gw;            // K / gw
-  int splits;        // K-splits (gridDim.z)
-  int gps;           // groups per split
+  int tiles_n, tiles_m, T;   // tiles (n fastest)
+  int S;             // K-stages (pairs of groups) per tile
+  int P;             // persistent CTAs (gridDim.x)
+  int streamk;       // 1: contiguous stage ranges per CTA; 0: whole tiles round-robin
   int sa_vec;        // sa rows readable as 16-byte vectors of 8 groups
   int sw_vec;        // sw rows readable as 16-byte vectors of 8 groups (gw == 128)
   const __half* sa;  // [M][G]
   const __half* sw;  // [N][Gw]
   __half* y;         // [M][N]
-  float* ws;         // [splits][M][N] fp32 partial outputs (splits > 1)
-  unsigned* counters;  // one arrival counter per output tile (splits > 1)
+  float* part;       // stream-K partial tiles [P][2][BT][128] fp32
+  unsigned* counters;  // [T] arrival counters of split tiles (zero between calls)
   int32_t* dump;     // [G][M][N] per-group partials (debug kernel only)
   unsigned long long wait_ns;
   int withhold;      // test hook: the producer never loads this stage (-1: off)
-  // Optional timeline trace (null: off), for the first trace_ctas CTAs (linear block id):
-  // SM clock stamps (clock64) [cta][role][step] with roles 0 producer issue and 1 converter
-  // done (per stage of two K-groups), 2 MMA issued and 3 epilogue done (per K-group);
+  // Optional timeline trace (null: off), for the first trace_ctas CTAs:
+  // SM clock stamps (clock64) [cta][role][step] with roles 0 producer issue, 1 converter
+  // done and 4 converter inputs ready (per stage of two K-groups), 2 MMA issued, 3
+  // epilogue done, 6 MMA inputs ready, 7 epilogue inputs ready, 8 MMA waits returned and
+  // 9 MMAs issued before their commits (per K-group);
   // [cta][5][0..1] = %globaltimer at start / end, [cta][5][2] = the SM the CTA ran on,
   // [cta][5][3] = clock64 at start.
   unsigned long long* trace;
@@ -70,35 +85,39 @@ struct GemmArgs {
 
 __device__ __forceinline__ void trace_stamp(const GemmArgs& a, int role, int step) {
   if (a.trace == nullptr) return;
-  const int cta = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+  const int cta = blockIdx.x;
   if (cta >= a.trace_ctas || step >= a.trace_steps) return;
-  a.trace[((size_t)cta * 6 + role) * a.trace_steps + step] =
+  a.trace[((size_t)cta * 10 + role) * a.trace_steps + step] =
       role == 5 ? globaltimer_ns() : clock_cycles();
 }
 
-template <int BT>
+template <int BT, int MODE>
 struct GemmCfg {
+  static constexpr bool AQ8 = MODE == MODE_AQ8;
   static constexpr int BM = 128;
   static constexpr int KPS = 2;                                    // K-groups per packed stage
-  static constexpr int NP = BT >= 128 ? 3 : 4;                     // packed stages
-  static constexpr int NX = 4;                                     // expanded operand slots
-  static constexpr int NSLOT = BT >= 128 ? 3 : (BT >= 64 ? 2 : 4);  // partial (D) slots
+  // operand slots (per group): weight columns in tensor memory + token tile in shared memory
+  static constexpr int NX = BT >= 128 ? (AQ8 ? 6 : 4) : 8;
+  static constexpr int NSLOT = BT >= 128 ? (AQ8 ? 2 : 3) : 4;     // partial (D) slots
   static constexpr int EPI_WARPS = BT >= 128 ? 8 : 4;
   static constexpr int CPT = BT >= 128 ? 64 : BT;  // columns per epilogue thread
+  static constexpr int CWG = BT >= 128 ? 1 : 2;    // converter warpgroups (alternate stages)
   static constexpr int CONV0 = 2;                  // first converter warp
-  static constexpr int EPI0 = 6;                   // first epilogue warp
+  static constexpr int EPI0 = CONV0 + 4 * CWG;     // first epilogue warp
   static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
-  static constexpr int MIN_BLOCKS = BT <= 32 ? 2 : 1;  // CTAs per SM the tile is sized for
   static constexpr int W_COL0 = 0;
   static constexpr int D_COL0 = NX * 32;
   static constexpr int TMEM_USED = D_COL0 + NSLOT * BT;
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
   static_assert(TMEM_USED <= 512, "tensor memory budget");
-  static constexpr int PKW = BM * 64 * KPS;   // [BM rows][128 B], 128-byte swizzle
-  static constexpr int PKA = BT * 64 * KPS;   // [BT rows][128 B], 128-byte swizzle
+  static constexpr int PKW = BM * 64 * KPS;              // [BM rows][128 B], 128-byte swizzle
+  static constexpr int PKA = AQ8 ? 0 : BT * 64 * KPS;   // [BT rows][128 B], 128-byte swizzle
   static constexpr int PK_STAGE = PKW + PKA;
-  static constexpr int XA = BT * 128;
+  static constexpr int XA = BT * 128;                    // one group's int8 token tile
   static constexpr int SAT = 2 * 8 * BT * 4;  // token scales: 2 blocks x [8 groups][BT] fp32
+  static constexpr int FIXED = NX * XA + SAT + 4096;
+  static constexpr int NP_FIT = (200 * 1024 - FIXED) / PK_STAGE;
+  static constexpr int NP = NP_FIT > 12 ? 12 : (NP_FIT < 2 ? 2 : NP_FIT);  // packed stages
   static constexpr int OFF_PK = 0;
   static constexpr int OFF_XA = OFF_PK + NP * PK_STAGE;
   static constexpr int OFF_SAT = OFF_XA + NX * XA;
@@ -113,17 +132,18 @@ struct GemmCfg {
 __device__ __forceinline__ uint32_t expand_lo(uint32_t w) { return (w << 4) & 0xF0F0F0F0u; }
 __device__ __forceinline__ uint32_t expand_hi(uint32_t w) { return w & 0xF0F0F0F0u; }
 
-// The 8 fp16 scales of groups gbeg .. gbeg+7 of one row, as raw bits (zeros from gend on).
-// vec: one 16-byte load (row offset + gbeg aligned to 8 elements, weight group == 128).
-// Otherwise element loads of base[row_off + g*128/gw].
+// The 8 fp16 scales of groups gbeg .. gbeg+7 of one row, as raw bits (zeros outside
+// [glo, ghi)).  vec: one 16-byte load (gbeg a multiple of 8, 16-byte aligned rows, weight
+// group == 128).  Otherwise element loads of base[row_off + g*128/gw].
 __device__ __forceinline__ uint4 load_scale_block(const __half* base, size_t row_off, int gbeg,
-                                                  int gend, bool vec, int gw) {
+                                                  int glo, int ghi, bool vec, int gw) {
   if (vec) return __ldg(reinterpret_cast<const uint4*>(base + row_off + gbeg));
   uint32_t h[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int g = gbeg + j;
-    h[j] = g < gend ? __half_as_ushort(base[row_off + (size_t)((g * 128) / gw)]) : 0u;
+    h[j] = (g >= glo && g < ghi) ? __half_as_ushort(base[row_off + (size_t)((g * 128) / gw)])
+                                 : 0u;
   }
   return make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
                     h[6] | (h[7] << 16));
@@ -134,11 +154,55 @@ __device__ __forceinline__ float half_of(const uint4& v, int j) {
   return __half2float(__ushort_as_half((uint16_t)((j & 1) ? (w >> 16) : (w & 0xFFFFu))));
 }
 
-template <int BT, bool DUMP>
-__global__ void __launch_bounds__(GemmCfg<BT>::THREADS, GemmCfg<BT>::MIN_BLOCKS)
+// ------------------------------------------------------------------ work distribution
+
+struct Seg {
+  int t;    // tile
+  int gb;   // first K-group
+  int ge;   // one past the last K-group
+};
+
+__device__ __forceinline__ long long sk_u0(const GemmArgs& a, int c) {
+  return (long long)c * a.T * a.S / a.P;
+}
+
+// CTA owning stage-unit u under the stream-K partition.
+__device__ __forceinline__ int sk_owner(const GemmArgs& a, long long u) {
+  const long long U = (long long)a.T * a.S;
+  return (int)(((u + 1) * a.P - 1) / U);
+}
+
+// k-th segment of this CTA; false when there is none.
+__device__ __forceinline__ bool get_seg(const GemmArgs& a, int k, Seg& sg) {
+  const int c = blockIdx.x;
+  if (!a.streamk) {
+    const int t = c + k * a.P;
+    if (t >= a.T) return false;
+    sg.t = t;
+    sg.gb = 0;
+    sg.ge = a.G;
+    return true;
+  }
+  const long long u0 = sk_u0(a, c), u1 = sk_u0(a, c + 1);
+  if (u0 >= u1) return false;
+  const int tf = (int)(u0 / a.S), tl = (int)((u1 - 1) / a.S);
+  const int t = tf + k;
+  if (t > tl) return false;
+  const int sb = t == tf ? (int)(u0 % a.S) : 0;
+  const int se = t == tl ? (int)((u1 - 1) % a.S) + 1 : a.S;
+  sg.t = t;
+  sg.gb = sb * 2;
+  sg.ge = min(se * 2, a.G);
+  return true;
+}
+
+template <int BT, int MODE>
+__global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmW,
                      const __grid_constant__ CUtensorMap tmA, const GemmArgs args) {
-  using C = GemmCfg<BT>;
+  using C = GemmCfg<BT, MODE>;
+  constexpr bool DUMP = MODE == MODE_DUMP;
+  constexpr bool AQ8 = C::AQ8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -160,11 +224,6 @@ __global__ void __launch_bounds__(GemmCfg<BT>::THREADS, GemmCfg<BT>::MIN_BLOCKS)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * C::BM;
-  const int m0 = blockIdx.y * BT;
-  const int g0 = blockIdx.z * args.gps;
-  const int ng = min(args.gps, args.G - g0);
-  const int ns = (ng + C::KPS - 1) / C::KPS;   // packed stages of this CTA
   const uint64_t lim = args.wait_ns;
 
   if (threadIdx.x == 0) {
@@ -202,253 +261,325 @@ __global__ void __launch_bounds__(GemmCfg<BT>::THREADS, GemmCfg<BT>::MIN_BLOCKS)
   volatile int* never = s_never;
   if (threadIdx.x == 0) {
     trace_stamp(args, 5, 0);
-    if (args.trace != nullptr && args.trace_steps > 3) {
+    if (args.trace != nullptr && args.trace_steps > 3 && (int)blockIdx.x < args.trace_ctas) {
       uint32_t smid;
       asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-      const int cta = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
-      if (cta < args.trace_ctas) {
-        args.trace[((size_t)cta * 6 + 5) * args.trace_steps + 2] = smid;
-        args.trace[((size_t)cta * 6 + 5) * args.trace_steps + 3] = clock_cycles();
-      }
+      args.trace[((size_t)blockIdx.x * 10 + 5) * args.trace_steps + 2] = smid;
+      args.trace[((size_t)blockIdx.x * 10 + 5) * args.trace_steps + 3] = clock_cycles();
     }
   }
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int last = -1;
-      for (int s = 0; s < ns; ++s) {
-        const int st = s % C::NP;
-        if (!mbar_wait(smem_u32(&pk_empty[st]), ((uint32_t)(s / C::NP) & 1u) ^ 1u, lim,
-                       abort_flag))
-          break;
-        if (s == args.withhold) continue;
-        const uint32_t fb = smem_u32(&pk_full[st]);
-        const int x = (g0 + s * C::KPS) * 64;   // byte column of the stage's first group
-        mbar_arrive_expect_tx(fb, C::PK_STAGE);
-        tma_load_2d(smem_u32(pk + st * C::PK_STAGE), &tmW, fb, x, n0);
-        tma_load_2d(smem_u32(pk + st * C::PK_STAGE + C::PKW), &tmA, fb, x, m0);
-        trace_stamp(args, 0, s);
-        last = s;
-      }
-      // Never leave the CTA with bulk copies in flight: wait for the last stages issued.
-      for (int s = (last - C::NP + 1 > 0 ? last - C::NP + 1 : 0); s <= last; ++s) {
-        if (s == args.withhold) continue;
-        mbar_wait(smem_u32(&pk_full[s % C::NP]), (uint32_t)(s / C::NP) & 1u, lim, never);
+    // The whole warp runs the loop (converged); lane 0 issues.
+    int q = 0, i = 0, last = -1;   // flat stage / group counters of this CTA
+    bool ok = true;
+    Seg sg;
+    for (int k = 0; ok && get_seg(args, k, sg); ++k) {
+      const int n0 = (sg.t % args.tiles_n) * C::BM;
+      const int m0 = (sg.t / args.tiles_n) * BT;
+      for (int g = sg.gb; g < sg.ge; g += C::KPS, ++q) {
+        const int nk = min(C::KPS, sg.ge - g);
+        const int st = q % C::NP;
+        ok = mbar_wait(smem_u32(&pk_empty[st]), ((uint32_t)(q / C::NP) & 1u) ^ 1u, lim,
+                       abort_flag);
+        if constexpr (AQ8) {   // the token tiles land in the operand slots themselves
+          for (int j = 0; j < nk && ok; ++j)
+            ok = mbar_wait(smem_u32(&x_empty[(i + j) % C::NX]),
+                           ((uint32_t)((i + j) / C::NX) & 1u) ^ 1u, lim, abort_flag);
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        if (q == args.withhold) {
+          i += nk;
+          continue;
+        }
+        if (lane == 0) {
+          const uint32_t fb = smem_u32(&pk_full[st]);
+          mbar_arrive_expect_tx(fb, C::PKW + (AQ8 ? nk * C::XA : C::PKA));
+          tma_load_2d(smem_u32(pk + st * C::PK_STAGE), &tmW, fb, g * 64, n0);
+          if constexpr (AQ8) {
+            for (int j = 0; j < nk; ++j)
+              tma_load_2d(smem_u32(xa + ((i + j) % C::NX) * C::XA), &tmA, fb, (g + j) * 128, m0);
+          } else {
+            tma_load_2d(smem_u32(pk + st * C::PK_STAGE + C::PKW), &tmA, fb, g * 64, m0);
+          }
+          trace_stamp(args, 0, q);
+        }
+        __syncwarp();
+        last = q;
+        i += nk;
       }
     }
+    // Never leave the CTA with bulk copies in flight: wait for the last stages issued.
+    for (int s = (last - C::NP + 1 > 0 ? last - C::NP + 1 : 0); s <= last; ++s) {
+      if (s == args.withhold) continue;
+      mbar_wait(smem_u32(&pk_full[s % C::NP]), (uint32_t)(s / C::NP) & 1u, lim, never);
+    }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(128, BT);
-      for (int i = 0; i < ng; ++i) {
+    // The whole warp runs the loop (converged); lane 0 issues the MMAs and commits.
+    constexpr uint32_t idesc = idesc_i8(128, BT);
+    int i = 0;
+    bool ok = true;
+    Seg sg;
+    for (int k = 0; ok && get_seg(args, k, sg); ++k) {
+      for (int g = sg.gb; g < sg.ge; ++g, ++i) {
         const int xs = i % C::NX;
         const int sl = i % C::NSLOT;
-        if (!mbar_wait(smem_u32(&x_full[xs]), (uint32_t)(i / C::NX) & 1u, lim, abort_flag)) break;
-        if (!mbar_wait(smem_u32(&d_empty[sl]), ((uint32_t)(i / C::NSLOT) & 1u) ^ 1u, lim,
-                       abort_flag))
-          break;
+        ok = mbar_wait(smem_u32(&x_full[xs]), (uint32_t)(i / C::NX) & 1u, lim, abort_flag) &&
+             mbar_wait(smem_u32(&d_empty[sl]), ((uint32_t)(i / C::NSLOT) & 1u) ^ 1u, lim,
+                       abort_flag);
+        if (lane == 0) trace_stamp(args, 8, i);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
         tc_fence_after();
-        const uint32_t a0 = tbase + C::W_COL0 + xs * 32;
-        const uint32_t d = tbase + C::D_COL0 + sl * BT;
-        const uint64_t b0 = smem_desc_k_sw128(smem_u32(xa + xs * C::XA));
+        if (lane == 0) {
+          trace_stamp(args, 6, i);
+          const uint32_t a0 = tbase + C::W_COL0 + xs * 32;
+          const uint32_t d = tbase + C::D_COL0 + sl * BT;
+          const uint64_t b0 = smem_desc_k_sw128(smem_u32(xa + xs * C::XA));
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          umma_i8_ts(d, a0 + j * 8, b0 + (uint64_t)(j * 2), idesc, j > 0 ? 1u : 0u);
-        umma_commit(smem_u32(&x_empty[xs]));
-        umma_commit(smem_u32(&d_full[sl]));
-        trace_stamp(args, 2, i);
+          for (int j = 0; j < 4; ++j)
+            umma_i8_ts(d, a0 + j * 8, b0 + (uint64_t)(j * 2), idesc, j > 0 ? 1u : 0u);
+          trace_stamp(args, 9, i);
+          umma_commit(smem_u32(&x_empty[xs]));
+          umma_commit(smem_u32(&d_full[sl]));
+          trace_stamp(args, 2, i);
+        }
+        __syncwarp();
       }
-      umma_commit(smem_u32(mma_done));
-      mbar_wait(smem_u32(mma_done), 0u, lim, never);
     }
-  } else if (warp >= C::CONV0 && warp < C::CONV0 + 4) {
+    if (lane == 0) umma_commit(smem_u32(mma_done));
+    __syncwarp();
+    mbar_wait(smem_u32(mma_done), 0u, lim, never);
+    __syncwarp();
+  } else if (warp >= C::CONV0 && warp < C::CONV0 + 4 * C::CWG) {
     // ------------------------------------------------------------ converters
+    // With two converter warpgroups, warpgroup w takes the stages q with q % 2 == w.
+    const int cwg = (warp - C::CONV0) >> 2;
     const int row = 32 * (warp & 3) + lane;            // this thread's TMEM lane = W row
-    const int ct = threadIdx.x - 32 * C::CONV0;        // 0..127, for the token rows
+    const int ct = threadIdx.x - 32 * (C::CONV0 + 4 * cwg);  // 0..127, for the token rows
     const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
-    constexpr int NIT = C::KPS * BT * 8 / 128;         // token 8-byte units per thread
-    for (int s = 0; s < ns; ++s) {
-      const int st = s % C::NP;
-      const int i0 = s * C::KPS;
-      const int nk = min(C::KPS, ng - i0);   // groups of this stage inside the split
-      bool ok = mbar_wait(smem_u32(&pk_full[st]), (uint32_t)(s / C::NP) & 1u, lim, abort_flag);
-      for (int j = 0; j < nk; ++j)
-        ok = ok && mbar_wait(smem_u32(&x_empty[(i0 + j) % C::NX]),
-                             ((uint32_t)((i0 + j) / C::NX) & 1u) ^ 1u, lim, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      const uint8_t* pw = pk + st * C::PK_STAGE;
-      const uint8_t* pa = pw + C::PKW;
-      // All shared-memory reads of the stage first, so their latencies overlap.
-      uint4 wraw[8];   // this thread's weight row: 16-byte chunk c sits at c ^ (row & 7)
+    constexpr int NIT = AQ8 ? 1 : C::KPS * BT * 8 / 128;   // token 8-byte units per thread
+    int q = 0, i = 0;
+    bool ok = true;
+    Seg sg;
+    for (int k = 0; ok && get_seg(args, k, sg); ++k) {
+      for (int g = sg.gb; g < sg.ge; g += C::KPS, ++q) {
+        const int st = q % C::NP;
+        const int nk = min(C::KPS, sg.ge - g);
+        if (q % C::CWG != cwg) {
+          i += nk;
+          continue;
+        }
+        ok = mbar_wait(smem_u32(&pk_full[st]), (uint32_t)(q / C::NP) & 1u, lim, abort_flag);
+        for (int j = 0; j < nk; ++j)
+          ok = ok && mbar_wait(smem_u32(&x_empty[(i + j) % C::NX]),
+                               ((uint32_t)((i + j) / C::NX) & 1u) ^ 1u, lim, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        if (lane == 0 && (warp & 3) == 2) trace_stamp(args, 4, q);
+        const uint8_t* pw = pk + st * C::PK_STAGE;
+        // All shared-memory reads of the stage first, so their latencies overlap.
+        uint4 wraw[8];   // this thread's weight row: 16-byte chunk c sits at c ^ (row & 7)
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        wraw[c] = *reinterpret_cast<const uint4*>(pw + row * 128 + ((c ^ (row & 7)) << 4));
-      uint2 araw[NIT];
+        for (int c = 0; c < 8; ++c)
+          wraw[c] = *reinterpret_cast<const uint4*>(pw + row * 128 + ((c ^ (row & 7)) << 4));
+        uint2 araw[NIT];
+        if constexpr (!AQ8) {
+          const uint8_t* pa = pw + C::PKW;
 #pragma unroll
-      for (int q = 0; q < NIT; ++q) {
-        const int it = ct + 128 * q;
-        const int j = it / (BT * 8), rem = it % (BT * 8);
-        const int r = rem >> 3, u = rem & 7;
-        araw[q] = *reinterpret_cast<const uint2*>(
-            pa + r * 128 + (((4 * j + (u >> 1)) ^ (r & 7)) << 4) + ((u & 1) << 3));
-      }
-#pragma unroll
-      for (int j = 0; j < C::KPS; ++j) {
-        if (j < nk) {
-          const int xs = (i0 + j) % C::NX;
-          uint32_t e0[16], e1[16];
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const uint4 a = wraw[4 * j + c], b = wraw[4 * j + 2 + c];
-            e0[8 * c + 0] = expand_lo(a.x); e0[8 * c + 1] = expand_hi(a.x);
-            e0[8 * c + 2] = expand_lo(a.y); e0[8 * c + 3] = expand_hi(a.y);
-            e0[8 * c + 4] = expand_lo(a.z); e0[8 * c + 5] = expand_hi(a.z);
-            e0[8 * c + 6] = expand_lo(a.w); e0[8 * c + 7] = expand_hi(a.w);
-            e1[8 * c + 0] = expand_lo(b.x); e1[8 * c + 1] = expand_hi(b.x);
-            e1[8 * c + 2] = expand_lo(b.y); e1[8 * c + 3] = expand_hi(b.y);
-            e1[8 * c + 4] = expand_lo(b.z); e1[8 * c + 5] = expand_hi(b.z);
-            e1[8 * c + 6] = expand_lo(b.w); e1[8 * c + 7] = expand_hi(b.w);
+          for (int x = 0; x < NIT; ++x) {
+            // unit v = row pair index: rows r and r+4 of an 8-row block share a load
+            // phase, and their 16-byte chunks fall in different banks
+            const int it = ct + 128 * x;
+            const int j = it / (BT * 8), rem = it % (BT * 8);
+            const int v = rem >> 3, u = rem & 7;
+            const int r = (v & ~7) | ((v & 1) << 2) | ((v >> 1) & 3);
+            araw[x] = *reinterpret_cast<const uint2*>(
+                pa + r * 128 + (((4 * j + (u >> 1)) ^ (r & 7)) << 4) + ((u & 1) << 3));
           }
-          const uint32_t tw = tbase + t_lane + C::W_COL0 + xs * 32;
-          tmem_st16(tw, e0);
-          tmem_st16(tw + 16, e1);
         }
-      }
 #pragma unroll
-      for (int q = 0; q < NIT; ++q) {
-        const int it = ct + 128 * q;
-        const int j = it / (BT * 8), rem = it % (BT * 8);
-        const int r = rem >> 3, u = rem & 7;
-        if (j < nk) {
-          uint4 o;
-          o.x = expand_lo(araw[q].x);
-          o.y = expand_hi(araw[q].x);
-          o.z = expand_lo(araw[q].y);
-          o.w = expand_hi(araw[q].y);
-          *reinterpret_cast<uint4*>(xa + ((i0 + j) % C::NX) * C::XA + r * 128 +
-                                    ((u ^ (r & 7)) << 4)) = o;
+        for (int j = 0; j < C::KPS; ++j) {
+          if (j < nk) {
+            const int xs = (i + j) % C::NX;
+            uint32_t e0[16], e1[16];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const uint4 a = wraw[4 * j + c], b = wraw[4 * j + 2 + c];
+              e0[8 * c + 0] = expand_lo(a.x); e0[8 * c + 1] = expand_hi(a.x);
+              e0[8 * c + 2] = expand_lo(a.y); e0[8 * c + 3] = expand_hi(a.y);
+              e0[8 * c + 4] = expand_lo(a.z); e0[8 * c + 5] = expand_hi(a.z);
+              e0[8 * c + 6] = expand_lo(a.w); e0[8 * c + 7] = expand_hi(a.w);
+              e1[8 * c + 0] = expand_lo(b.x); e1[8 * c + 1] = expand_hi(b.x);
+              e1[8 * c + 2] = expand_lo(b.y); e1[8 * c + 3] = expand_hi(b.y);
+              e1[8 * c + 4] = expand_lo(b.z); e1[8 * c + 5] = expand_hi(b.z);
+              e1[8 * c + 6] = expand_lo(b.w); e1[8 * c + 7] = expand_hi(b.w);
+            }
+            const uint32_t tw = tbase + t_lane + C::W_COL0 + xs * 32;
+            tmem_st16(tw, e0);
+            tmem_st16(tw + 16, e1);
+          }
         }
+        if constexpr (!AQ8) {
+#pragma unroll
+          for (int x = 0; x < NIT; ++x) {
+            const int it = ct + 128 * x;
+            const int j = it / (BT * 8), rem = it % (BT * 8);
+            const int v = rem >> 3, u = rem & 7;
+            const int r = (v & ~7) | ((v & 1) << 2) | ((v >> 1) & 3);
+            if (j < nk) {
+              uint4 o;
+              o.x = expand_lo(araw[x].x);
+              o.y = expand_hi(araw[x].x);
+              o.z = expand_lo(araw[x].y);
+              o.w = expand_hi(araw[x].y);
+              *reinterpret_cast<uint4*>(xa + ((i + j) % C::NX) * C::XA + r * 128 +
+                                        ((u ^ (r & 7)) << 4)) = o;
+            }
+          }
+          fence_proxy_async_smem();
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(smem_u32(&pk_empty[st]));
+          for (int j = 0; j < nk; ++j) mbar_arrive(smem_u32(&x_full[(i + j) % C::NX]));
+        }
+        if (lane == 0 && (warp & 3) == 2) trace_stamp(args, 1, q);
+        i += nk;
       }
-      tmem_st_wait();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(smem_u32(&pk_empty[st]));
-        for (int j = 0; j < nk; ++j) mbar_arrive(smem_u32(&x_full[(i0 + j) % C::NX]));
-      }
-      if (threadIdx.x == 32 * C::CONV0) trace_stamp(args, 1, s);
     }
   } else if (warp >= C::EPI0) {
     // ------------------------------------------------------------ epilogue
     const int et = threadIdx.x - 32 * C::EPI0;
     const int h = (warp - C::EPI0) >> 2;           // column block (64 columns) of this warp
     const int row = 32 * (warp & 3) + lane;        // TMEM lane = weight row in the tile
-    const int n = n0 + row;
-    const bool nvalid = n < args.N;
-    const int mt = m0 + et;                        // token whose scales this thread fetches
-    const bool tvalid = et < BT && mt < args.M;
     const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
     constexpr int NE = C::EPI_WARPS * 32;
     const int M = args.M, N = args.N;
-    // One weight group spans this CTA's whole K-range: sw factors out of the sum.
-    const bool hoist = (g0 * 128) / args.gw == ((g0 + ng - 1) * 128) / args.gw;
-    const int nblk = (ng + 7) / 8;
     const bool sa_vec = args.sa_vec != 0, sw_vec = args.sw_vec != 0;
 
-    auto sa_block = [&](int b) -> uint4 {
-      if (DUMP || !tvalid) return make_uint4(0, 0, 0, 0);
-      return load_scale_block(args.sa, (size_t)mt * args.G, g0 + 8 * b, g0 + ng, sa_vec, 128);
-    };
-    auto sw_block = [&](int b) -> uint4 {
-      if (DUMP || !nvalid) return make_uint4(0, 0, 0, 0);
-      return load_scale_block(args.sw, (size_t)n * args.Gw, g0 + 8 * b, g0 + ng, sw_vec,
-                              args.gw);
+    // Scales of the 8-group block starting at gb8 of segment sg (this thread's token / row).
+    auto block_scales = [&](const Seg& sg, int gb8, uint4& sa, uint4& sw) {
+      sa = make_uint4(0, 0, 0, 0);
+      sw = make_uint4(0, 0, 0, 0);
+      if (DUMP) return;
+      const int mt = (sg.t / args.tiles_n) * BT + et;
+      const int nn = (sg.t % args.tiles_n) * C::BM + row;
+      if (et < BT && mt < M)
+        sa = load_scale_block(args.sa, (size_t)mt * args.G, gb8, sg.gb, sg.ge, sa_vec, 128);
+      if (nn < N)
+        sw = load_scale_block(args.sw, (size_t)nn * args.Gw, gb8, sg.gb, sg.ge, sw_vec, args.gw);
     };
 
     float2 acc[C::CPT / 2];
-#pragma unroll
-    for (int e = 0; e < C::CPT / 2; ++e) acc[e] = make_float2(0.0f, 0.0f);
-    float sw_hoisted = 0.0f;
-
-    uint4 sa_c = sa_block(0), sw_c = sw_block(0);
     bool ok = true, aborted = false;
-    for (int b = 0; b < nblk; ++b) {
-      uint4 sa_n = make_uint4(0, 0, 0, 0), sw_n = make_uint4(0, 0, 0, 0);
-      if (b + 1 < nblk) {   // the next block's scales are in flight during this block
-        sa_n = sa_block(b + 1);
-        sw_n = sw_block(b + 1);
-      }
-      float* sat = s_sat + (b & 1) * 8 * BT;
-      if (et < BT) {
+    int i = 0;     // flat group counter of this CTA
+    int buf = 0;   // token-scale buffer in use
+    Seg sg, nx;
+    bool have = get_seg(args, 0, sg);
+    uint4 sa_c = make_uint4(0, 0, 0, 0), sw_c = make_uint4(0, 0, 0, 0);
+    if (have) block_scales(sg, sg.gb & ~7, sa_c, sw_c);
+    for (int k = 0; have && !aborted; ++k) {
+      const int n0 = (sg.t % args.tiles_n) * C::BM;
+      const int m0 = (sg.t / args.tiles_n) * BT;
+      const int n = n0 + row;
+      const bool nvalid = n < N;
+      // One weight group spans the whole segment: sw factors out of the sum.
+      const bool hoist = (sg.gb * 128) / args.gw == ((sg.ge - 1) * 128) / args.gw;
+      const bool have_next = get_seg(args, k + 1, nx);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) sat[j * BT + et] = half_of(sa_c, j);
-      }
-      aborted = bar_red_or(1, NE, !ok);   // token scales visible; one abort decision for all
-      if (aborted) break;
-      if (b == 0) sw_hoisted = half_of(sw_c, 0) * (1.0f / 256.0f);
+      for (int e = 0; e < C::CPT / 2; ++e) acc[e] = make_float2(0.0f, 0.0f);
+      float sw_hoisted = 0.0f;
+      for (int gb8 = sg.gb & ~7; gb8 < sg.ge; gb8 += 8) {
+        // the next block's scales are in flight while this block is processed
+        uint4 sa_n, sw_n;
+        if (gb8 + 8 < sg.ge)
+          block_scales(sg, gb8 + 8, sa_n, sw_n);
+        else if (have_next)
+          block_scales(nx, nx.gb & ~7, sa_n, sw_n);
+        else
+          sa_n = sw_n = make_uint4(0, 0, 0, 0);
+        float* sat = s_sat + buf * 8 * BT;
+        if (et < BT) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) sat[j * BT + et] = half_of(sa_c, j);
+        }
+        aborted = bar_red_or(1, NE, !ok);   // token scales visible; one abort decision
+        if (aborted) break;
+        if (gb8 <= sg.gb) sw_hoisted = half_of(sw_c, sg.gb - gb8) * (1.0f / 256.0f);
+        const int jb = max(sg.gb - gb8, 0), je = min(sg.ge - gb8, 8);
 #pragma unroll 1
-      for (int j = 0; j < 8; ++j) {
-        const int i = 8 * b + j;
-        if (i >= ng || !ok) break;
-        const int sl = i % C::NSLOT;
-        ok = mbar_wait(smem_u32(&d_full[sl]), (uint32_t)(i / C::NSLOT) & 1u, lim, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        const float4* sab = reinterpret_cast<const float4*>(sat + j * BT + h * 64);
-        const float swj = half_of(sw_c, j) * (1.0f / 256.0f);
-        const float2 sw2 = make_float2(swj, swj);
-        const uint32_t td = tbase + t_lane + C::D_COL0 + sl * BT + h * 64;
+        for (int j = jb; j < je; ++j, ++i) {
+          const int sl = i % C::NSLOT;
+          ok = mbar_wait(smem_u32(&d_full[sl]), (uint32_t)(i / C::NSLOT) & 1u, lim, abort_flag);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          if (et == 0) trace_stamp(args, 7, i);
+          tc_fence_after();
+          const float4* sab = reinterpret_cast<const float4*>(sat + j * BT + h * 64);
+          const float swj = half_of(sw_c, j) * (1.0f / 256.0f);
+          const float2 sw2 = make_float2(swj, swj);
+          const uint32_t td = tbase + t_lane + C::D_COL0 + sl * BT + h * 64;
 #pragma unroll
-        for (int cc = 0; cc < C::CPT / 16; ++cc) {
-          uint32_t p[16];
-          tmem_ld16(td + cc * 16, p);
-          if constexpr (DUMP) {
-            const int g = g0 + i;
+          for (int cc = 0; cc < C::CPT / 16; ++cc) {
+            uint32_t p[16];
+            tmem_ld16(td + cc * 16, p);
+            if constexpr (DUMP) {
+              const int g = gb8 + j;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int m = m0 + h * 64 + cc * 16 + e;
-              if (m < M && nvalid)
-                args.dump[((size_t)g * M + m) * N + n] = static_cast<int32_t>(p[e]) >> 8;
-            }
-          } else {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const float4 s4 = sab[cc * 4 + q];
-              const float2 pa = make_float2((float)(int32_t)p[4 * q + 0], (float)(int32_t)p[4 * q + 1]);
-              const float2 pb = make_float2((float)(int32_t)p[4 * q + 2], (float)(int32_t)p[4 * q + 3]);
-              float2 sa_a = make_float2(s4.x, s4.y), sa_b = make_float2(s4.z, s4.w);
-              if (!hoist) {
-                sa_a = __fmul2_rn(sa_a, sw2);
-                sa_b = __fmul2_rn(sa_b, sw2);
+              for (int e = 0; e < 16; ++e) {
+                const int m = m0 + h * 64 + cc * 16 + e;
+                if (m < M && nvalid)
+                  args.dump[((size_t)g * M + m) * N + n] = static_cast<int32_t>(p[e]) >> 8;
               }
-              acc[cc * 8 + 2 * q] = __ffma2_rn(pa, sa_a, acc[cc * 8 + 2 * q]);
-              acc[cc * 8 + 2 * q + 1] = __ffma2_rn(pb, sa_b, acc[cc * 8 + 2 * q + 1]);
+            } else {
+#pragma unroll
+              for (int qq = 0; qq < 4; ++qq) {
+                const float4 s4 = sab[cc * 4 + qq];
+                const float2 pa =
+                    make_float2((float)(int32_t)p[4 * qq + 0], (float)(int32_t)p[4 * qq + 1]);
+                const float2 pb =
+                    make_float2((float)(int32_t)p[4 * qq + 2], (float)(int32_t)p[4 * qq + 3]);
+                float2 sa_a = make_float2(s4.x, s4.y), sa_b = make_float2(s4.z, s4.w);
+                if (!hoist) {
+                  sa_a = __fmul2_rn(sa_a, sw2);
+                  sa_b = __fmul2_rn(sa_b, sw2);
+                }
+                acc[cc * 8 + 2 * qq] = __ffma2_rn(pa, sa_a, acc[cc * 8 + 2 * qq]);
+                acc[cc * 8 + 2 * qq + 1] = __ffma2_rn(pb, sa_b, acc[cc * 8 + 2 * qq + 1]);
+              }
             }
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(smem_u32(&d_empty[sl]));
+            if (et == 0) trace_stamp(args, 3, i);
+          }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(smem_u32(&d_empty[sl]));
-          if (et == 0) trace_stamp(args, 3, i);
-        }
+        buf ^= 1;
+        sa_c = sa_n;
+        sw_c = sw_n;
       }
-      sa_c = sa_n;
-      sw_c = sw_n;
-    }
-    if (!aborted) aborted = bar_red_or(1, NE, !ok);
-
-    if constexpr (!DUMP) {
-      if (!aborted) {
+      // ---- segment finished: write the tile, or hand its partial to the fixup
+      aborted = aborted || bar_red_or(1, NE, !ok);
+      if (aborted) break;
+      if constexpr (!DUMP) {
         if (hoist) {
           const float2 sh = make_float2(sw_hoisted, sw_hoisted);
 #pragma unroll
           for (int e = 0; e < C::CPT / 2; ++e) acc[e] = __fmul2_rn(acc[e], sh);
         }
-        if (args.splits == 1) {
+        const long long tu0 = (long long)sg.t * args.S;
+        const int cf = args.streamk ? sk_owner(args, tu0) : (int)blockIdx.x;
+        const int cl = args.streamk ? sk_owner(args, tu0 + args.S - 1) : (int)blockIdx.x;
+        if (cf == cl) {
 #pragma unroll
           for (int e = 0; e < C::CPT; ++e) {
             const int m = m0 + h * 64 + e;
@@ -456,37 +587,39 @@ __global__ void __launch_bounds__(GemmCfg<BT>::THREADS, GemmCfg<BT>::MIN_BLOCKS)
             if (m < M && nvalid) args.y[(size_t)m * N + n] = __float2half_rn(v);
           }
         } else {
-          float* wsp = args.ws + (size_t)blockIdx.z * M * N;
+          // partial slot: 0 for this CTA's first tile, 1 for its last (a CTA shares at most
+          // those two tiles with other CTAs)
+          auto slot_of = [&](int c) -> size_t {
+            const int tf = (int)(sk_u0(args, c) / args.S);
+            return ((size_t)c * 2 + (sg.t == tf ? 0 : 1)) * (size_t)(BT * C::BM);
+          };
+          float* mine = args.part + slot_of(blockIdx.x);
 #pragma unroll
           for (int e = 0; e < C::CPT; ++e) {
-            const int m = m0 + h * 64 + e;
-            const float v = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
-            if (m < M && nvalid) wsp[(size_t)m * N + n] = v;
+            const int ml = h * 64 + e;
+            mine[(size_t)ml * C::BM + row] = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
           }
           __threadfence();
           bar_red_or(1, NE, false);
-          const int tile = blockIdx.y * gridDim.x + blockIdx.x;
           if (et == 0) {
-            const unsigned old = atomicAdd(&args.counters[tile], 1u);
-            *reinterpret_cast<volatile int*>(s_last) = (old == (unsigned)args.splits - 1u);
+            const unsigned old = atomicAdd(&args.counters[sg.t], 1u);
+            *reinterpret_cast<volatile int*>(s_last) = (old == (unsigned)(cl - cf));
           }
           bar_red_or(1, NE, false);
           if (*reinterpret_cast<volatile int*>(s_last)) {
             __threadfence();
-            // Sum the splits in split order (deterministic), 16 columns at a time with all
-            // of a split's loads issued before they are added.
+            // the contributions, added in CTA order whoever arrives last
 #pragma unroll
             for (int e0 = 0; e0 < C::CPT; e0 += 16) {
               float sum[16];
 #pragma unroll
               for (int e = 0; e < 16; ++e) sum[e] = 0.0f;
-              for (int z = 0; z < args.splits; ++z) {
+              for (int c = cf; c <= cl; ++c) {
+                const float* src = args.part + slot_of(c);
                 float v[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                  const int m = m0 + h * 64 + e0 + e;
-                  v[e] = (m < M && nvalid) ? __ldcg(args.ws + ((size_t)z * M + m) * N + n) : 0.0f;
-                }
+                for (int e = 0; e < 16; ++e)
+                  v[e] = __ldcg(src + (size_t)(h * 64 + e0 + e) * C::BM + row);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) sum[e] += v[e];
               }
@@ -496,10 +629,12 @@ __global__ void __launch_bounds__(GemmCfg<BT>::THREADS, GemmCfg<BT>::MIN_BLOCKS)
                 if (m < M && nvalid) args.y[(size_t)m * N + n] = __float2half_rn(sum[e]);
               }
             }
-            if (et == 0) atomicExch(&args.counters[tile], 0u);
+            if (et == 0) atomicExch(&args.counters[sg.t], 0u);
           }
         }
       }
+      have = have_next;
+      sg = nx;
     }
   }
 

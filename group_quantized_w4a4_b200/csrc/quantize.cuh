@@ -47,9 +47,18 @@ __device__ __forceinline__ uint32_t quant_pack8(const uint4& v, float sf) {
   return out;
 }
 
+// The same 8 values as 16*q in signed bytes, in the GEMM's operand order: bytes 0..3 hold
+// elements 0,2,4,6 and bytes 4..7 elements 1,3,5,7 (what the GEMM makes of a packed word).
+__device__ __forceinline__ uint2 quant_expand8(const uint4& v, float sf) {
+  const uint32_t w = quant_pack8(v, sf);
+  return make_uint2((w << 4) & 0xF0F0F0F0u, w & 0xF0F0F0F0u);
+}
+
 // CH > 0: the group is exactly CH 128-wide chunks, kept in registers (one pass over HBM).
 // CH == 0: any group width; absmax pass then quantize pass (the second pass hits L2).
-template <int CH>
+// EXP: write the expanded operand form ([rows][K] bytes of 16*q, see quant_expand8)
+// instead of packed nibbles ([rows][K/2] bytes).
+template <int CH, bool EXP = false>
 __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __restrict__ x,
                                                             int64_t rows, int64_t K, int group,
                                                             uint8_t* __restrict__ packed,
@@ -71,6 +80,7 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __rest
     const uint4* src = reinterpret_cast<const uint4*>(x + row * K + g * group) + lane16;
     uint32_t* dst =
         reinterpret_cast<uint32_t*>(packed + row * (K / 2) + g * (group / 2)) + lane16;
+    uint2* xdst = reinterpret_cast<uint2*>(packed + row * K + (int64_t)g * group) + lane16;
 
     float amax = 0.0f;
     if constexpr (CH > 0) {
@@ -87,7 +97,12 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __rest
       const float sf = __half2float(s);
       if (live) {
 #pragma unroll
-        for (int c = 0; c < CH; ++c) dst[c * 16] = quant_pack8(v[c], sf);
+        for (int c = 0; c < CH; ++c) {
+          if constexpr (EXP)
+            xdst[c * 16] = quant_expand8(v[c], sf);
+          else
+            dst[c * 16] = quant_pack8(v[c], sf);
+        }
         if (lane16 == 0) scales[row * G + g] = s;
       }
     } else {
@@ -101,7 +116,12 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __rest
       const __half s = __float2half_rn(__fdiv_rn(amax, 7.0f));
       const float sf = __half2float(s);
       if (live) {
-        for (int c = 0; c < chunks; ++c) dst[c * 16] = quant_pack8(__ldg(src + c * 16), sf);
+        for (int c = 0; c < chunks; ++c) {
+          if constexpr (EXP)
+            xdst[c * 16] = quant_expand8(__ldg(src + c * 16), sf);
+          else
+            dst[c * 16] = quant_pack8(__ldg(src + c * 16), sf);
+        }
         if (lane16 == 0) scales[row * G + g] = s;
       }
     }

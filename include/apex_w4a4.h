@@ -64,6 +64,29 @@ apex_status_t apex_quantize_act_int4(const void *x_f16, int64_t M, int64_t K, in
                                      void *x_packed_u8, void *x_scales_f16, void *stream);
 
 /*
+ * Online activation quantization into the GEMM's expanded operand form (same rule and the
+ * same q and scales as apex_quantize_act_int4; group_a must be 128).  x_q8 [M][K] bytes:
+ * for every 8 consecutive elements k0..k7 of a row, bytes 0..3 hold 16*q(k0), 16*q(k2),
+ * 16*q(k4), 16*q(k6) and bytes 4..7 hold 16*q(k1), 16*q(k3), 16*q(k5), 16*q(k7), as signed
+ * 8-bit integers -- the values are still 4-bit; this is the order the tensor-core path
+ * consumes, so the GEMM need not unpack activations.  Twice the bytes of the packed form;
+ * worth it when M is large (prefill), where activation traffic is small next to the math.
+ * x_q8 8-byte aligned (16 for the GEMM), x_scales_f16 [M][K/128].
+ */
+apex_status_t apex_quantize_act_int4_expanded(const void *x_f16, int64_t M, int64_t K,
+                                              int32_t group_a, void *x_q8, void *x_scales_f16,
+                                              void *stream);
+
+/*
+ * The W4A4 GEMM on expanded activations (from apex_quantize_act_int4_expanded): the same
+ * result, arguments and rules as apex_w4a4_gemm, with a_q8 [M][K] in place of a_packed.
+ */
+apex_status_t apex_w4a4_gemm_expanded(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                      int32_t group_w, const void *a_q8, const void *a_scales,
+                                      const void *w_packed, const void *w_scales, void *y_f16,
+                                      void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * The W4A4 GEMM: y_f16[M][N] = fp16_rne(sum_g P_g * sa * sw), accumulated in fp32.
  *   a_packed [M][K/2], a_scales [M][K/group_a]   (from apex_quantize_act_int4)
  *   w_packed [N][K/2], w_scales [N][K/group_w]   (from apex_pack_weights_int4)
@@ -141,10 +164,13 @@ void apex_debug_withhold_step(int32_t step);
 
 /*
  * Tracing hook: the next apex_w4a4_gemm launch on this host thread writes timestamps for
- * its first `ctas` CTAs (linear block id) into the device buffer trace[ctas][6][steps]
+ * its first `ctas` CTAs (persistent CTA index) into the device buffer trace[ctas][10][steps]
  * (uint64).  SM clock cycles (clock64): [c][0][s] producer issued stage s (a pair of
  * K-groups), [c][1][s] converters done with stage s, [c][2][i] MMAs of K-group i issued,
- * [c][3][i] epilogue done with K-group i, [c][4][i] scales of K-group i loaded;
+ * [c][3][i] epilogue done with K-group i, [c][4][s] converter inputs of stage s ready,
+ * [c][6][i] MMA inputs of K-group i ready (after the tensor-core fence), [c][7][i]
+ * epilogue inputs of K-group i ready, [c][8][i] MMA waits returned, [c][9][i] MMAs of
+ * K-group i issued before their commits;
  * [c][5][0] / [c][5][1] %globaltimer (ns) at CTA start / end, [c][5][2] the SM it ran on,
  * [c][5][3] clock64 at CTA start.  Steps beyond `steps` are not recorded.
  */

@@ -273,6 +273,68 @@ def test_gemm_large_workloads_sampled_rows(apex, name):
     assert_close(got, ref)
 
 
+# ------------------------------------------------------------------ expanded activations
+
+
+def expected_expanded(q):
+    """16*q in the GEMM operand order: per 8 elements, k0,k2,k4,k6 then k1,k3,k5,k7."""
+    rows, K = q.shape
+    blk = q.reshape(rows, K // 8, 8)
+    order = blk[:, :, [0, 2, 4, 6, 1, 3, 5, 7]] * 16
+    return order.reshape(rows, K).astype(np.int8).view(np.uint8)
+
+
+@pytest.mark.parametrize("rows,K,dist", [(16, 512, "normal"), (130, 2048, "outlier"),
+                                         (1, 128, "student_t")])
+def test_quantize_expanded_bit_exact(apex, rows, K, dist):
+    x = synth.activations(rows, K, dist, 17 + rows)
+    ap_ref, sa_ref = oracle.quantize_pack(x, 128)
+    q8, sa = apex.quantize_act_expanded(dev(x), 128)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(q8), expected_expanded(oracle.unpack(ap_ref, K).astype(np.int64)))
+    assert np.array_equal(f16(sa), sa_ref.view(np.uint16))
+
+
+def run_gemm_expanded(apex, x, wp, sw, M, N, K, gw):
+    q8, sa = apex.quantize_act_expanded(dev(x), 128)
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    w = apex.workspace(M, N, K, 128, gw)
+    apex.apex_w4a4_gemm_expanded(M, N, K, 128, gw, q8, sa, dev(wp), dev(sw), y, w)
+    torch.cuda.synchronize()
+    check_status(apex)
+    return host(y).astype(np.float64)
+
+
+@pytest.mark.parametrize("M,N,K,gw", [(16, 256, 512, 128), (130, 257, 1024, 128),
+                                      (256, 384, 2048, 512), (200, 128, 768, 768),
+                                      (129, 1024, 4096, 128)])
+def test_gemm_expanded_matches_oracle(apex, M, N, K, gw):
+    a = synth.activations(M, K, "outlier", 3 * M + K)
+    w = synth.weights(N, K, N + 3 * K)
+    ap, sa = oracle.quantize_pack(a, 128)
+    wp, sw = oracle.quantize_pack(w, gw)
+    ref = oracle.gemm(ap, sa, wp, sw, M, N, K, 128, gw)
+    assert_close(run_gemm_expanded(apex, a, wp, sw, M, N, K, gw), ref)
+
+
+@pytest.mark.parametrize("name", ["prefill_m4096_n8192_k8192", "mlp_down_m2048_n8192_k28672",
+                                  "sweep_m1024_gw512"])
+def test_gemm_expanded_large_sampled_rows(apex, name):
+    g = synth.workloads()[name]
+    a, w = synth.make(g)
+    wp, sw = apex.pack_weights(dev(w), g.gw)
+    q8, sa = apex.quantize_act_expanded(dev(a), 128)
+    y = torch.empty((g.M, g.N), dtype=torch.float16, device="cuda")
+    ws = apex.workspace(g.M, g.N, g.K, 128, g.gw)
+    apex.apex_w4a4_gemm_expanded(g.M, g.N, g.K, 128, g.gw, q8, sa, wp, sw, y, ws)
+    torch.cuda.synchronize()
+    check_status(apex)
+    rows = np.array(sorted({0, 1, 127, 128, g.M // 3, g.M - 1}), dtype=np.int64)
+    ap_ref, sa_ref = oracle.quantize_pack(a[rows], 128)
+    ref = oracle.gemm(ap_ref, sa_ref, host(wp), host(sw), rows.size, g.N, g.K, 128, g.gw)
+    assert_close(host(y)[rows].astype(np.float64), ref)
+
+
 # ------------------------------------------------------------------ failure path
 
 

@@ -28,7 +28,7 @@ def apex():
     return m
 
 
-@pytest.mark.parametrize("M,N,K,gw", [(16, 2048, 8192, 128), (48, 1024, 4096, 512),
+@pytest.mark.parametrize("M,N,K,gw", [(16, 2048, 8192, 128), (32, 1024, 4096, 512),
                                       (16, 256, 512, 128)])
 def test_noalloc_matches_workspace_gemm_twice(apex, M, N, K, gw):
     a = synth.activations(M, K, "normal", 70 + M)
