@@ -149,10 +149,14 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ the apex arm
 
+EXPANDED_MIN_M = 128   # from this many tokens on, the step uses the expanded activation form
+
+
 class Problem:
     """Device-resident operands for one workload, in C copies (inputs larger than L2)."""
 
     def __init__(self, apex, torch, g: synth.Gemm, copies: int):
+        self.expanded = g.M >= EXPANDED_MIN_M
         self.g = g
         a, w = synth.make(g)
         self.a_host = a
@@ -167,7 +171,8 @@ class Problem:
             self.x.append(a_d if c == 0 else a_d.clone())
             self.wp.append(wp0 if c == 0 else wp0.clone())
             self.sw.append(sw0 if c == 0 else sw0.clone())
-            self.ap.append(torch.empty((g.M, g.K // 2), dtype=torch.uint8, device=dev))
+            self.ap.append(torch.empty((g.M, g.K if self.expanded else g.K // 2),
+                                       dtype=torch.uint8, device=dev))
             self.sa.append(torch.empty((g.M, g.K // 128), dtype=torch.float16, device=dev))
         self.y = torch.empty((g.M, g.N), dtype=torch.float16, device=dev)
         self.ws = apex.workspace(g.M, g.N, g.K, 128, g.gw)
@@ -187,11 +192,14 @@ def apex_step(apex, p: Problem, i: int, stream, ev=None):
     c = i % p.copies
     if ev is not None:
         ev[0].record(stream)
-    apex.apex_quantize_act_int4(p.x[c], g.M, g.K, 128, p.ap[c], p.sa[c], stream)
+    if p.expanded:
+        apex.apex_quantize_act_int4_expanded(p.x[c], g.M, g.K, 128, p.ap[c], p.sa[c], stream)
+    else:
+        apex.apex_quantize_act_int4(p.x[c], g.M, g.K, 128, p.ap[c], p.sa[c], stream)
     if ev is not None:
         ev[1].record(stream)
-    apex.apex_w4a4_gemm(g.M, g.N, g.K, 128, g.gw, p.ap[c], p.sa[c], p.wp[c], p.sw[c], p.y,
-                        p.ws, None, stream)
+    gemm = apex.apex_w4a4_gemm_expanded if p.expanded else apex.apex_w4a4_gemm
+    gemm(g.M, g.N, g.K, 128, g.gw, p.ap[c], p.sa[c], p.wp[c], p.sw[c], p.y, p.ws, None, stream)
     if ev is not None:
         ev[2].record(stream)
 
@@ -340,6 +348,7 @@ def run_apex(args, rank, world, local):
         extra[SECOND_WORKLOAD] = {
             "value": round(world * g2.ops / (ms2 * 1e-3) / 1e12, 2), "unit": "TOPS",
             "ms_per_step": round(ms2, 4),
+            "activation_form": "expanded" if g2.M >= EXPANDED_MIN_M else "packed",
             "quantize_ms": round(statistics.mean(qm2), 5),
             "roofline": roofline_obj(g2, statistics.mean(gm2), peaks, peaks_kind)}
         del p2
@@ -353,6 +362,7 @@ def run_apex(args, rank, world, local):
         "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights, fp16)",
         "config": {"workload": g.name, "M": g.M, "N": g.N, "K": g.K, "group_a": 128,
                    "group_w": g.gw, "parallelism": f"replicas x{world}",
+                   "activation_form": "expanded" if g.M >= EXPANDED_MIN_M else "packed",
                    "l2": f"inputs larger than L2: {p_copies(g, l2)} rotating copies"},
         "roofline": roofline_obj(g, gemm_avg, peaks, peaks_kind),
         "e2e": {"value": round(world * g.ops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
