@@ -187,42 +187,37 @@ def copies_for(g: synth.Gemm, l2_bytes: int) -> int:
     return c
 
 
-def apex_step(apex, p: Problem, i: int, stream, ev=None):
-    g = p.g
-    c = i % p.copies
-    if ev is not None:
-        ev[0].record(stream)
+def apex_quantize(apex, p: Problem, i: int, stream):
+    g, c = p.g, i % p.copies
     if p.expanded:
         apex.apex_quantize_act_int4_expanded(p.x[c], g.M, g.K, 128, p.ap[c], p.sa[c], stream)
     else:
         apex.apex_quantize_act_int4(p.x[c], g.M, g.K, 128, p.ap[c], p.sa[c], stream)
-    if ev is not None:
-        ev[1].record(stream)
+
+
+def apex_gemm(apex, p: Problem, i: int, stream):
+    g, c = p.g, i % p.copies
     gemm = apex.apex_w4a4_gemm_expanded if p.expanded else apex.apex_w4a4_gemm
     gemm(g.M, g.N, g.K, 128, g.gw, p.ap[c], p.sa[c], p.wp[c], p.sw[c], p.y, p.ws, None, stream)
-    if ev is not None:
-        ev[2].record(stream)
 
 
-def time_workload(apex, torch, g, steps, warmup, world, l2_bytes, clocks=None):
-    """W eager warm-up steps, then exactly K steps replayed from one CUDA graph (captured
-    beforehand, so the timed region has no host launch overhead), CUDA events around
-    every kernel inside the graph."""
-    p = Problem(apex, torch, g, copies_for(g, l2_bytes))
-    for i in range(warmup):
-        apex_step(apex, p, i, torch.cuda.current_stream())
-    torch.cuda.synchronize()
-    if apex.apex_get_device_status() != 0:
-        raise RuntimeError("device status not clean after warm-up")
-    # external=True: captured as real event-record nodes, so they time the replay
-    evs = [tuple(torch.cuda.Event(enable_timing=True, external=True) for _ in range(3))
-           for _ in range(steps)]
+def apex_step(apex, p: Problem, i: int, stream):
+    """One step of the hot path: online activation quantize, then the W4A4 GEMM."""
+    apex_quantize(apex, p, i, stream)
+    apex_gemm(apex, p, i, stream)
+
+
+def timed_graph(torch, fn, steps, first, world, clocks=None):
+    """Capture fn(i, stream) for i = first .. first+steps-1 in one CUDA graph, then replay it
+    once between CUDA events on the capturing stream (barrier + synchronize on both sides).
+    Kernels follow each other with no event in between, so each launch overlaps the tail of
+    the previous one as it does in a real stream.  Returns (total ms, clock record)."""
     side = torch.cuda.Stream()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.stream(side):
         with torch.cuda.graph(graph, stream=side):
             for i in range(steps):
-                apex_step(apex, p, warmup + i, side, evs[i])
+                fn(first + i, side)
     torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -236,13 +231,29 @@ def time_workload(apex, torch, g, steps, warmup, world, l2_bytes, clocks=None):
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop() if clocks else None
+    del graph
+    return start.elapsed_time(stop), clk
+
+
+def time_workload(apex, torch, g, steps, warmup, world, l2_bytes, clocks=None):
+    """W eager warm-up steps, then three timed CUDA-graph replays of exactly K launches each:
+    the K steps (quantize + GEMM; the headline), the K GEMMs alone and the K quantizer
+    launches alone (per-kernel average durations for the roofline)."""
+    p = Problem(apex, torch, g, copies_for(g, l2_bytes))
+    stream = torch.cuda.current_stream()
+    for i in range(max(warmup, p.copies)):   # every copy's quantized operands exist
+        apex_step(apex, p, i, stream)
+    torch.cuda.synchronize()
+    if apex.apex_get_device_status() != 0:
+        raise RuntimeError("device status not clean after warm-up")
+    step = lambda i, s: apex_step(apex, p, i, s)
+    total_ms, clk = timed_graph(torch, step, steps, warmup, world, clocks)
+    gemm_ms, _ = timed_graph(torch, lambda i, s: apex_gemm(apex, p, i, s), steps, warmup, world)
+    quant_ms, _ = timed_graph(torch, lambda i, s: apex_quantize(apex, p, i, s), steps, warmup,
+                              world)
     if apex.apex_get_device_status() != 0:
         raise RuntimeError("device status not clean after the timed steps")
-    total_ms = start.elapsed_time(stop)
-    quant_ms = [e0.elapsed_time(e1) for e0, e1, _ in evs]
-    gemm_ms = [e1.elapsed_time(e2) for _, e1, e2 in evs]
-    del graph
-    return p, total_ms, gemm_ms, clk, quant_ms
+    return p, total_ms, gemm_ms / steps, clk, quant_ms / steps
 
 
 def e2e_workload(apex, torch, g, steps, warmup, p: Problem):
@@ -330,10 +341,10 @@ def run_apex(args, rank, world, local):
     peaks, peaks_kind = load_peaks()
     g = synth.workloads()[args.workload]
     clocks = ClockSampler(local) if rank == 0 else None
-    p, total_ms, gemm_ms, clk, quant_ms = time_workload(apex, torch, g, args.steps,
-                                                        args.warmup, world, l2, clocks)
+    p, total_ms, gemm_avg, clk, quant_avg = time_workload(apex, torch, g, args.steps,
+                                                          args.warmup, world, l2, clocks)
     ms_step = max_over_ranks(total_ms / args.steps, world)
-    gemm_avg = statistics.mean(gemm_ms)
+    gemm_avg = max_over_ranks(gemm_avg, world)
     value = world * g.ops / (ms_step * 1e-3) / 1e12
     e2e_ms, hb, db = e2e_workload(apex, torch, g, max(3, args.steps), args.warmup, p)
     e2e_ms = max_over_ranks(e2e_ms, world)
@@ -344,13 +355,14 @@ def run_apex(args, rank, world, local):
         g2 = synth.workloads()[SECOND_WORKLOAD]
         p2, tot2, gm2, _, qm2 = time_workload(apex, torch, g2, max(3, args.steps // 4),
                                               args.warmup, world, l2)
+        gm2, qm2 = max_over_ranks(gm2, world), max_over_ranks(qm2, world)
         ms2 = max_over_ranks(tot2 / max(3, args.steps // 4), world)
         extra[SECOND_WORKLOAD] = {
             "value": round(world * g2.ops / (ms2 * 1e-3) / 1e12, 2), "unit": "TOPS",
             "ms_per_step": round(ms2, 4),
             "activation_form": "expanded" if g2.M >= EXPANDED_MIN_M else "packed",
-            "quantize_ms": round(statistics.mean(qm2), 5),
-            "roofline": roofline_obj(g2, statistics.mean(gm2), peaks, peaks_kind)}
+            "quantize_ms": round(qm2, 5), "gemm_ms": round(gm2, 5),
+            "roofline": roofline_obj(g2, gm2, peaks, peaks_kind)}
         del p2
     if rank != 0:
         return None
@@ -369,11 +381,12 @@ def run_apex(args, rank, world, local):
                 "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db,
                 "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": 2 * args.steps,
-        "launch": "one CUDA graph of the K timed steps (eager warm-up)",
-        "quantize": {"kernel_ms": round(statistics.mean(quant_ms), 5),
-                     "bytes": g.quant_bytes(),
-                     "GB/s": round(g.quant_bytes() / (statistics.mean(quant_ms) * 1e-3) / 1e9,
-                                   1)},
+        "launch": ("one CUDA graph of the K timed steps (eager warm-up), kernels launched as "
+                   "programmatic dependents; per-kernel times from two more graphs of K "
+                   "launches of that kernel alone"),
+        "gemm": {"kernel_ms": round(gemm_avg, 5), "bytes": g.gemm_bytes()},
+        "quantize": {"kernel_ms": round(quant_avg, 5), "bytes": g.quant_bytes(),
+                     "GB/s": round(g.quant_bytes() / (quant_avg * 1e-3) / 1e9, 1)},
         "clocks": clk,
         "impl": "apex",
     }

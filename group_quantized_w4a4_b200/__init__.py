@@ -214,8 +214,8 @@ def apex_debug_withhold_step(step: int):
 
 
 def apex_debug_trace_next_gemm(trace, ctas: int, steps: int):
-    """trace: int64 CUDA tensor with at least ctas*10*steps elements (zeroed by the caller)."""
-    if trace.numel() < ctas * 10 * steps:
+    """trace: int64 CUDA tensor with at least ctas*16*steps elements (zeroed by the caller)."""
+    if trace.numel() < ctas * 16 * steps:
         raise ValueError("trace buffer too small")
     load_library().apex_debug_trace_next_gemm(_ptr(trace), int(ctas), int(steps))
 

@@ -143,6 +143,10 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, bool allow_streamk) {
     p.streamk = 1;
     const long long units = (long long)p.T * p.S;
     p.P = units < sms ? (int)units : sms;
+    if ((long long)p.P * units >= (1ll << 31)) {   // the device partition math is 32-bit
+      p.streamk = 0;
+      p.P = p.T < sms ? p.T : sms;
+    }
   }
   return p;
 }
@@ -168,14 +172,39 @@ struct Maps {
   CUtensorMap w, a;
 };
 
+// Every kernel is launched as a programmatic dependent of the previous work in the stream,
+// so its launch and prologue overlap that work's tail (each kernel waits for the previous
+// grid before its first global access).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                       cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 template <int BT, int MODE>
 apex_status_t launch_bt(const Plan& p, const Maps& m, const GemmArgs& a, cudaStream_t s) {
   using C = GemmCfg<BT, MODE>;
   auto kern = apex::w4a4_gemm_kernel<BT, MODE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (e != cudaSuccess) return APEX_ERR_CUDA;
-  kern<<<p.P, C::THREADS, C::SMEM, s>>>(m.w, m.a, a);
-  return cuda_status(cudaPeekAtLastError());
+  static thread_local int attr_dev = -1;   // the attribute is per device; set it once each
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return APEX_ERR_CUDA;
+  if (attr_dev != dev) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+        cudaSuccess)
+      return APEX_ERR_CUDA;
+    attr_dev = dev;
+  }
+  return cuda_status(launch_pdl(kern, (unsigned)p.P, C::THREADS, (size_t)C::SMEM, s, m.w, m.a, a));
 }
 
 template <int MODE>
@@ -202,6 +231,7 @@ GemmArgs base_args(const Plan& p, int64_t M, int64_t N, int64_t K, int32_t gw,
   a.tiles_m = p.tiles_m;
   a.T = p.T;
   a.S = p.S;
+  a.TS = p.streamk ? p.T * p.S : 0;
   a.P = p.P;
   a.streamk = p.streamk;
   // Scales are fetched in 16-byte blocks of 8 groups when rows are 16-byte strided.
@@ -238,18 +268,22 @@ apex_status_t quantize_launch(const void* x, int64_t rows, int64_t K, int32_t gr
   const __half* xh = static_cast<const __half*>(x);
   uint8_t* pk = static_cast<uint8_t*>(packed);
   __half* sc = static_cast<__half*>(scales);
+  const unsigned nb = (unsigned)blocks;
+  cudaError_t e;
   if (expanded) {
     if (group != 128) return APEX_ERR_UNSUPPORTED;
-    apex::quantize_pack_kernel<1, true><<<(unsigned)blocks, threads, 0, s>>>(xh, rows, K, group, pk,
-                                                                             sc);
-  } else if (group == 128)
-    apex::quantize_pack_kernel<1><<<(unsigned)blocks, threads, 0, s>>>(xh, rows, K, group, pk, sc);
-  else if (group == 256)
-    apex::quantize_pack_kernel<2><<<(unsigned)blocks, threads, 0, s>>>(xh, rows, K, group, pk, sc);
-  else if (group == 512)
-    apex::quantize_pack_kernel<4><<<(unsigned)blocks, threads, 0, s>>>(xh, rows, K, group, pk, sc);
-  else
-    apex::quantize_pack_kernel<0><<<(unsigned)blocks, threads, 0, s>>>(xh, rows, K, group, pk, sc);
+    e = launch_pdl(apex::quantize_pack_kernel<1, true>, nb, threads, 0, s, xh, rows, K, group,
+                   pk, sc);
+  } else if (group == 128) {
+    e = launch_pdl(apex::quantize_pack_kernel<1>, nb, threads, 0, s, xh, rows, K, group, pk, sc);
+  } else if (group == 256) {
+    e = launch_pdl(apex::quantize_pack_kernel<2>, nb, threads, 0, s, xh, rows, K, group, pk, sc);
+  } else if (group == 512) {
+    e = launch_pdl(apex::quantize_pack_kernel<4>, nb, threads, 0, s, xh, rows, K, group, pk, sc);
+  } else {
+    e = launch_pdl(apex::quantize_pack_kernel<0>, nb, threads, 0, s, xh, rows, K, group, pk, sc);
+  }
+  if (e != cudaSuccess) return APEX_ERR_CUDA;
   return cuda_status(cudaPeekAtLastError());
 }
 

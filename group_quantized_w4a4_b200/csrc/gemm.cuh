@@ -23,10 +23,11 @@
 //               one [BT x 128 B] int8 tile per group straight into the MMA operand slot.
 //   warp 1      MMA issuer (one thread): 4 x tcgen05.mma kind::i8 (K = 32 each) per group
 //               into a tensor-memory slot; one exact int32 partial per group.
-//   warps 2..   converters (one warpgroup, or two taking alternate stages for narrow
-//               tiles): nibbles -> int8 in registers.  The weight row of each thread goes to
-//               tensor memory (tcgen05.st); packed token rows go to shared memory in the
-//               128-byte-swizzled K-major operand layout.
+//   warps 2..   converters (one warpgroup; for narrow tiles two, each taking one of the
+//               two K-groups of every stage): nibbles -> int8 in registers.  The weight row
+//               of each thread goes to tensor memory (tcgen05.st) for wide tiles, or to
+//               shared memory for narrow ones; packed token rows go to shared memory.  Both
+//               shared-memory operands use the 128-byte-swizzled K-major layout.
 //   then        epilogue: tcgen05.ld of a group's partials while the next groups' MMAs
 //               run, fp32 scale by sa*sw and accumulate in registers (packed f32x2 math);
 //               fp16 output.  Each epilogue thread also fetches the scales it needs, one
@@ -59,6 +60,7 @@ struct GemmArgs {
   int Gw;            // K / gw
   int tiles_n, tiles_m, T;   // tiles (n fastest)
   int S;             // K-stages (pairs of groups) per tile
+  int TS;            // T * S
   int P;             // persistent CTAs (gridDim.x)
   int streamk;       // 1: contiguous stage ranges per CTA; 0: whole tiles round-robin
   int sa_vec;        // sa rows readable as 16-byte vectors of 8 groups
@@ -77,28 +79,45 @@ struct GemmArgs {
   // epilogue done, 6 MMA inputs ready, 7 epilogue inputs ready, 8 MMA waits returned and
   // 9 MMAs issued before their commits (per K-group);
   // [cta][5][0..1] = %globaltimer at start / end, [cta][5][2] = the SM the CTA ran on,
-  // [cta][5][3] = clock64 at start.
+  // [cta][5][3] = clock64 at start, [cta][5][4..5] = producer loop entry / first segment.
   unsigned long long* trace;
   int trace_ctas;
   int trace_steps;
 };
 
+constexpr int kTraceRoles = 16;
+
+// clock64 into trace slot [cta][role][step] (used for the prologue marks of role 5).
+__device__ __forceinline__ void trace_stamp_at(const GemmArgs& a, int role, int step) {
+  if (a.trace == nullptr) return;
+  const int cta = blockIdx.x;
+  if (cta >= a.trace_ctas || step >= a.trace_steps) return;
+  a.trace[((size_t)cta * kTraceRoles + role) * a.trace_steps + step] = clock_cycles();
+}
+
 __device__ __forceinline__ void trace_stamp(const GemmArgs& a, int role, int step) {
   if (a.trace == nullptr) return;
   const int cta = blockIdx.x;
   if (cta >= a.trace_ctas || step >= a.trace_steps) return;
-  a.trace[((size_t)cta * 10 + role) * a.trace_steps + step] =
+  a.trace[((size_t)cta * kTraceRoles + role) * a.trace_steps + step] =
       role == 5 ? globaltimer_ns() : clock_cycles();
 }
+
+#ifndef APEX_WSM_MAX_BT
+#define APEX_WSM_MAX_BT 0
+#endif
 
 template <int BT, int MODE>
 struct GemmCfg {
   static constexpr bool AQ8 = MODE == MODE_AQ8;
+  // Narrow tiles keep the expanded weight tile in shared memory (both MMA operands from
+  // shared memory); wide tiles keep it in tensor memory.
+  static constexpr bool WSM = !AQ8 && BT <= APEX_WSM_MAX_BT;
   static constexpr int BM = 128;
   static constexpr int KPS = 2;                                    // K-groups per packed stage
-  // operand slots (per group): weight columns in tensor memory + token tile in shared memory
-  static constexpr int NX = BT >= 128 ? (AQ8 ? 6 : 4) : 8;
-  static constexpr int NSLOT = BT >= 128 ? (AQ8 ? 2 : 3) : 4;     // partial (D) slots
+  // operand slots (per group): expanded weight tile (tensor or shared memory) + token tile
+  static constexpr int NX = WSM ? (BT <= 32 ? 6 : 4) : BT >= 128 ? (AQ8 ? 6 : 4) : 8;
+  static constexpr int NSLOT = WSM ? NX : BT >= 128 ? (AQ8 ? 2 : 3) : 4;  // partial (D) slots
   static constexpr int EPI_WARPS = BT >= 128 ? 8 : 4;
   static constexpr int CPT = BT >= 128 ? 64 : BT;  // columns per epilogue thread
   static constexpr int CWG = BT >= 128 ? 1 : 2;    // converter warpgroups (alternate stages)
@@ -106,7 +125,7 @@ struct GemmCfg {
   static constexpr int EPI0 = CONV0 + 4 * CWG;     // first epilogue warp
   static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
   static constexpr int W_COL0 = 0;
-  static constexpr int D_COL0 = NX * 32;
+  static constexpr int D_COL0 = WSM ? 0 : NX * 32;
   static constexpr int TMEM_USED = D_COL0 + NSLOT * BT;
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
   static_assert(TMEM_USED <= 512, "tensor memory budget");
@@ -114,18 +133,36 @@ struct GemmCfg {
   static constexpr int PKA = AQ8 ? 0 : BT * 64 * KPS;   // [BT rows][128 B], 128-byte swizzle
   static constexpr int PK_STAGE = PKW + PKA;
   static constexpr int XA = BT * 128;                    // one group's int8 token tile
+  static constexpr int XW = WSM ? BM * 128 : 0;          // one group's int8 weight tile
   static constexpr int SAT = 2 * 8 * BT * 4;  // token scales: 2 blocks x [8 groups][BT] fp32
-  static constexpr int FIXED = NX * XA + SAT + 4096;
+  static constexpr int FIXED = NX * (XA + XW) + SAT + 4096;
   static constexpr int NP_FIT = (200 * 1024 - FIXED) / PK_STAGE;
   static constexpr int NP = NP_FIT > 12 ? 12 : (NP_FIT < 2 ? 2 : NP_FIT);  // packed stages
   static constexpr int OFF_PK = 0;
   static constexpr int OFF_XA = OFF_PK + NP * PK_STAGE;
-  static constexpr int OFF_SAT = OFF_XA + NX * XA;
+  static constexpr int OFF_XW = OFF_XA + NX * XA;
+  static constexpr int OFF_SAT = OFF_XW + NX * XW;
   static constexpr int OFF_BAR = OFF_SAT + SAT;
-  static constexpr int NBAR = 2 * NP + 2 * NX + 2 * NSLOT + 1;
+  // Hand-off unit: the groups that pass between converters, MMA and epilogue under one
+  // barrier phase -- a whole stage for narrow tiles (the MMA issue loop is short on work
+  // per group there), a single group for wide ones (whose partial slots fill TMEM).
+  static constexpr int GPB = BT <= 64 ? KPS : 1;
+  static constexpr int NXU = NX / GPB;      // operand hand-off units in flight
+  static constexpr int NDU = NSLOT / GPB;   // partial hand-off units in flight
+  static_assert(NX % GPB == 0 && NSLOT % GPB == 0, "slots come in whole units");
+  static_assert(GPB == 1 || CWG * (KPS / CWG) == KPS, "converter split");
+  static constexpr int NBAR = 2 * NP + 2 * NXU + NDU + 1;
+  // one MMA-completion barrier per operand unit also tells the epilogue that the unit's
+  // partials are ready, which needs every partial slot to be reused no sooner than its
+  // operand slot
+  static_assert(NDU <= NXU, "partial units cannot outnumber operand units");
+  // operand slot of group j of stage q (flat group index gi)
+  static __device__ __forceinline__ int slot(int q, int gi, int j) {
+    return GPB == 1 ? gi % NX : (q % NXU) * GPB + j;
+  }
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
-  static_assert(PK_STAGE % 1024 == 0 && XA % 1024 == 0, "stage alignment");
+  static_assert(PK_STAGE % 1024 == 0 && XA % 1024 == 0 && XW % 1024 == 0, "stage alignment");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
@@ -162,14 +199,15 @@ struct Seg {
   int ge;   // one past the last K-group
 };
 
-__device__ __forceinline__ long long sk_u0(const GemmArgs& a, int c) {
-  return (long long)c * a.T * a.S / a.P;
+// First stage-unit of CTA c under the stream-K partition (32-bit: the host only picks
+// stream-K when P * T * S < 2^31).
+__device__ __forceinline__ int sk_u0(const GemmArgs& a, int c) {
+  return (int)((unsigned)c * (unsigned)a.TS / (unsigned)a.P);
 }
 
 // CTA owning stage-unit u under the stream-K partition.
-__device__ __forceinline__ int sk_owner(const GemmArgs& a, long long u) {
-  const long long U = (long long)a.T * a.S;
-  return (int)(((u + 1) * a.P - 1) / U);
+__device__ __forceinline__ int sk_owner(const GemmArgs& a, int u) {
+  return (int)((((unsigned)u + 1u) * (unsigned)a.P - 1u) / (unsigned)a.TS);
 }
 
 // k-th segment of this CTA; false when there is none.
@@ -183,13 +221,13 @@ __device__ __forceinline__ bool get_seg(const GemmArgs& a, int k, Seg& sg) {
     sg.ge = a.G;
     return true;
   }
-  const long long u0 = sk_u0(a, c), u1 = sk_u0(a, c + 1);
+  const int u0 = sk_u0(a, c), u1 = sk_u0(a, c + 1);
   if (u0 >= u1) return false;
-  const int tf = (int)(u0 / a.S), tl = (int)((u1 - 1) / a.S);
+  const int tf = u0 / a.S, tl = (u1 - 1) / a.S;
   const int t = tf + k;
   if (t > tl) return false;
-  const int sb = t == tf ? (int)(u0 % a.S) : 0;
-  const int se = t == tl ? (int)((u1 - 1) % a.S) + 1 : a.S;
+  const int sb = t == tf ? u0 - tf * a.S : 0;
+  const int se = t == tl ? (u1 - 1) - tl * a.S + 1 : a.S;
   sg.t = t;
   sg.gb = sb * 2;
   sg.ge = min(se * 2, a.G);
@@ -208,14 +246,16 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* pk = smem + C::OFF_PK;
   uint8_t* xa = smem + C::OFF_XA;
+  uint8_t* xw = smem + C::OFF_XW;
   float* s_sat = reinterpret_cast<float*>(smem + C::OFF_SAT);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* pk_full = bars;
   uint64_t* pk_empty = pk_full + C::NP;
   uint64_t* x_full = pk_empty + C::NP;
-  uint64_t* x_empty = x_full + C::NX;
-  uint64_t* d_full = x_empty + C::NX;
-  uint64_t* d_empty = d_full + C::NSLOT;
+  // g_done[s]: the MMAs of the group in operand slot s have completed -- its operand slot
+  // is free again and its partial is in tensor memory (one commit serves both waiters)
+  uint64_t* g_done = x_full + C::NXU;
+  uint64_t* d_empty = g_done + C::NXU;
   uint64_t* mma_done = d_empty + C::NSLOT;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* s_abort = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
@@ -226,17 +266,20 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
   const int lane = threadIdx.x & 31;
   const uint64_t lim = args.wait_ns;
 
+  if (threadIdx.x == 0 && args.trace != nullptr && (int)blockIdx.x < args.trace_ctas &&
+      args.trace_steps > 6)
+    args.trace[((size_t)blockIdx.x * kTraceRoles + 5) * args.trace_steps + 6] = globaltimer_ns();
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NP; ++i) {
       mbar_init(smem_u32(&pk_full[i]), 1);
-      mbar_init(smem_u32(&pk_empty[i]), 4);          // one arrival per converter warp
+      mbar_init(smem_u32(&pk_empty[i]), 4 * C::CWG);  // one arrival per converter warp
     }
-    for (int i = 0; i < C::NX; ++i) {
-      mbar_init(smem_u32(&x_full[i]), 4);
-      mbar_init(smem_u32(&x_empty[i]), 1);
+    for (int i = 0; i < C::NXU; ++i) {
+      // one arrival per converter warp that fills the unit
+      mbar_init(smem_u32(&x_full[i]), C::GPB == 1 ? 4 : 4 * C::CWG);
+      mbar_init(smem_u32(&g_done[i]), 1);
     }
-    for (int i = 0; i < C::NSLOT; ++i) {
-      mbar_init(smem_u32(&d_full[i]), 1);
+    for (int i = 0; i < C::NDU; ++i) {
       mbar_init(smem_u32(&d_empty[i]), C::EPI_WARPS);  // one arrival per epilogue warp
     }
     mbar_init(smem_u32(mma_done), 1);
@@ -256,6 +299,10 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Launched as a programmatic dependent: the prologue above overlaps the previous grid's
+  // tail; no global memory is read or written before that grid has completed.
+  grid_dep_wait();
+  grid_dep_launch();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(s_tmem);
   volatile int* abort_flag = s_abort;
   volatile int* never = s_never;
@@ -264,8 +311,8 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
     if (args.trace != nullptr && args.trace_steps > 3 && (int)blockIdx.x < args.trace_ctas) {
       uint32_t smid;
       asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-      args.trace[((size_t)blockIdx.x * 10 + 5) * args.trace_steps + 2] = smid;
-      args.trace[((size_t)blockIdx.x * 10 + 5) * args.trace_steps + 3] = clock_cycles();
+      args.trace[((size_t)blockIdx.x * kTraceRoles + 5) * args.trace_steps + 2] = smid;
+      args.trace[((size_t)blockIdx.x * kTraceRoles + 5) * args.trace_steps + 3] = clock_cycles();
     }
   }
 
@@ -275,18 +322,26 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
     int q = 0, i = 0, last = -1;   // flat stage / group counters of this CTA
     bool ok = true;
     Seg sg;
+    if (lane == 0) trace_stamp_at(args, 5, 4);
     for (int k = 0; ok && get_seg(args, k, sg); ++k) {
+      if (lane == 0 && k == 0) trace_stamp_at(args, 5, 5);
       const int n0 = (sg.t % args.tiles_n) * C::BM;
       const int m0 = (sg.t / args.tiles_n) * BT;
       for (int g = sg.gb; g < sg.ge; g += C::KPS, ++q) {
         const int nk = min(C::KPS, sg.ge - g);
         const int st = q % C::NP;
-        ok = mbar_wait(smem_u32(&pk_empty[st]), ((uint32_t)(q / C::NP) & 1u) ^ 1u, lim,
-                       abort_flag);
+        const uint32_t pe_par = ((uint32_t)(q / C::NP) & 1u) ^ 1u;
         if constexpr (AQ8) {   // the token tiles land in the operand slots themselves
-          for (int j = 0; j < nk && ok; ++j)
-            ok = mbar_wait(smem_u32(&x_empty[(i + j) % C::NX]),
-                           ((uint32_t)((i + j) / C::NX) & 1u) ^ 1u, lim, abort_flag);
+          const int u0 = C::GPB == 1 ? i : q;   // the stage's first hand-off unit
+          ok = mbar_wait2(smem_u32(&pk_empty[st]), pe_par, smem_u32(&g_done[u0 % C::NXU]),
+                          ((uint32_t)(u0 / C::NXU) & 1u) ^ 1u, lim, abort_flag);
+          if constexpr (C::GPB == 1) {
+            for (int j = 1; j < nk && ok; ++j)
+              ok = mbar_wait(smem_u32(&g_done[(i + j) % C::NXU]),
+                             ((uint32_t)((i + j) / C::NXU) & 1u) ^ 1u, lim, abort_flag);
+          }
+        } else {
+          ok = mbar_wait(smem_u32(&pk_empty[st]), pe_par, lim, abort_flag);
         }
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
@@ -300,7 +355,8 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
           tma_load_2d(smem_u32(pk + st * C::PK_STAGE), &tmW, fb, g * 64, n0);
           if constexpr (AQ8) {
             for (int j = 0; j < nk; ++j)
-              tma_load_2d(smem_u32(xa + ((i + j) % C::NX) * C::XA), &tmA, fb, (g + j) * 128, m0);
+              tma_load_2d(smem_u32(xa + C::slot(q, i + j, j) * C::XA), &tmA, fb, (g + j) * 128,
+                          m0);
           } else {
             tma_load_2d(smem_u32(pk + st * C::PK_STAGE + C::PKW), &tmA, fb, g * 64, m0);
           }
@@ -321,34 +377,50 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs the loop (converged); lane 0 issues the MMAs and commits.
     constexpr uint32_t idesc = idesc_i8(128, BT);
-    int i = 0;
+    int i = 0, q = 0;   // flat group / stage counters of this CTA
     bool ok = true;
     Seg sg;
     for (int k = 0; ok && get_seg(args, k, sg); ++k) {
-      for (int g = sg.gb; g < sg.ge; ++g, ++i) {
-        const int xs = i % C::NX;
-        const int sl = i % C::NSLOT;
-        ok = mbar_wait(smem_u32(&x_full[xs]), (uint32_t)(i / C::NX) & 1u, lim, abort_flag) &&
-             mbar_wait(smem_u32(&d_empty[sl]), ((uint32_t)(i / C::NSLOT) & 1u) ^ 1u, lim,
-                       abort_flag);
-        if (lane == 0) trace_stamp(args, 8, i);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        if (lane == 0) {
-          trace_stamp(args, 6, i);
-          const uint32_t a0 = tbase + C::W_COL0 + xs * 32;
-          const uint32_t d = tbase + C::D_COL0 + sl * BT;
-          const uint64_t b0 = smem_desc_k_sw128(smem_u32(xa + xs * C::XA));
+      for (int g = sg.gb; ok && g < sg.ge; g += C::KPS, ++q) {
+        const int nk = min(C::KPS, sg.ge - g);
+        // the stage's hand-off units: one per group, or the whole stage
+        for (int j0 = 0; j0 < nk; j0 += C::GPB) {
+          const int u = C::GPB == 1 ? i + j0 : q;
+          const int nu = min(C::GPB, nk - j0);
+          const int xu = u % C::NXU, du = u % C::NDU;
+          ok = mbar_wait2(smem_u32(&x_full[xu]), (uint32_t)(u / C::NXU) & 1u,
+                          smem_u32(&d_empty[du]), ((uint32_t)(u / C::NDU) & 1u) ^ 1u, lim,
+                          abort_flag);
+          if (lane == 0) trace_stamp(args, 8, i + j0);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          if (lane == 0) {
+            trace_stamp(args, 6, i + j0);
+            for (int t = 0; t < nu; ++t) {
+              const int xs = xu * C::GPB + t;
+              const uint32_t d = tbase + C::D_COL0 + (du * C::GPB + t) * BT;
+              const uint64_t b0 = smem_desc_k_sw128(smem_u32(xa + xs * C::XA));
+              if constexpr (C::WSM) {
+                const uint64_t a0 = smem_desc_k_sw128(smem_u32(xw + xs * C::XW));
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            umma_i8_ts(d, a0 + j * 8, b0 + (uint64_t)(j * 2), idesc, j > 0 ? 1u : 0u);
-          trace_stamp(args, 9, i);
-          umma_commit(smem_u32(&x_empty[xs]));
-          umma_commit(smem_u32(&d_full[sl]));
-          trace_stamp(args, 2, i);
+                for (int j = 0; j < 4; ++j)
+                  umma_i8_ss(d, a0 + (uint64_t)(j * 2), b0 + (uint64_t)(j * 2), idesc,
+                             j > 0 ? 1u : 0u);
+              } else {
+                const uint32_t a0 = tbase + C::W_COL0 + xs * 32;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  umma_i8_ts(d, a0 + j * 8, b0 + (uint64_t)(j * 2), idesc, j > 0 ? 1u : 0u);
+              }
+            }
+            trace_stamp(args, 9, i + j0);
+            umma_commit(smem_u32(&g_done[xu]));
+            trace_stamp(args, 2, i + j0);
+          }
+          __syncwarp();
         }
-        __syncwarp();
+        i += nk;
       }
     }
     if (lane == 0) umma_commit(smem_u32(mma_done));
@@ -357,12 +429,14 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
     __syncwarp();
   } else if (warp >= C::CONV0 && warp < C::CONV0 + 4 * C::CWG) {
     // ------------------------------------------------------------ converters
-    // With two converter warpgroups, warpgroup w takes the stages q with q % 2 == w.
+    // Warpgroup w expands the K-groups j of every stage with j % CWG == w, so with two
+    // warpgroups both work on each stage at once, one group each.
     const int cwg = (warp - C::CONV0) >> 2;
-    const int row = 32 * (warp & 3) + lane;            // this thread's TMEM lane = W row
+    const int row = 32 * (warp & 3) + lane;            // this thread's W row (TMEM lane)
     const int ct = threadIdx.x - 32 * (C::CONV0 + 4 * cwg);  // 0..127, for the token rows
     const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
-    constexpr int NIT = AQ8 ? 1 : C::KPS * BT * 8 / 128;   // token 8-byte units per thread
+    constexpr int JPW = C::KPS / C::CWG;                   // groups per warpgroup per stage
+    constexpr int NITG = AQ8 ? 0 : BT * 8 / 128;           // token 8-byte units per thread
     int q = 0, i = 0;
     bool ok = true;
     Seg sg;
@@ -370,46 +444,80 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
       for (int g = sg.gb; g < sg.ge; g += C::KPS, ++q) {
         const int st = q % C::NP;
         const int nk = min(C::KPS, sg.ge - g);
-        if (q % C::CWG != cwg) {
-          i += nk;
-          continue;
+        // the stage's bytes, and the operand slots it fills.  With whole-stage units every
+        // converter warp waits for the unit's previous use (even a warpgroup with no group
+        // in a short stage), so its arrival can only count toward this use.
+        const uint32_t pf_par = (uint32_t)(q / C::NP) & 1u;
+        if constexpr (C::GPB != 1) {
+          ok = mbar_wait2(smem_u32(&pk_full[st]), pf_par, smem_u32(&g_done[q % C::NXU]),
+                          ((uint32_t)(q / C::NXU) & 1u) ^ 1u, lim, abort_flag);
+        } else {
+          ok = cwg < nk ? mbar_wait2(smem_u32(&pk_full[st]), pf_par,
+                                     smem_u32(&g_done[(i + cwg) % C::NXU]),
+                                     ((uint32_t)((i + cwg) / C::NXU) & 1u) ^ 1u, lim, abort_flag)
+                        : mbar_wait(smem_u32(&pk_full[st]), pf_par, lim, abort_flag);
+#pragma unroll
+          for (int jj = 1; jj < JPW; ++jj) {
+            const int j = cwg + C::CWG * jj;
+            if (j < nk)
+              ok = ok && mbar_wait(smem_u32(&g_done[(i + j) % C::NXU]),
+                                   ((uint32_t)((i + j) / C::NXU) & 1u) ^ 1u, lim, abort_flag);
+          }
         }
-        ok = mbar_wait(smem_u32(&pk_full[st]), (uint32_t)(q / C::NP) & 1u, lim, abort_flag);
-        for (int j = 0; j < nk; ++j)
-          ok = ok && mbar_wait(smem_u32(&x_empty[(i + j) % C::NX]),
-                               ((uint32_t)((i + j) / C::NX) & 1u) ^ 1u, lim, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         if (lane == 0 && (warp & 3) == 2) trace_stamp(args, 4, q);
         const uint8_t* pw = pk + st * C::PK_STAGE;
-        // All shared-memory reads of the stage first, so their latencies overlap.
-        uint4 wraw[8];   // this thread's weight row: 16-byte chunk c sits at c ^ (row & 7)
+        // All shared-memory reads first, so their latencies overlap.  Packed W row: the
+        // 16-byte chunk c of the 128-byte stage row sits at c ^ (row & 7); group j owns
+        // chunks 4j .. 4j+3.
+        uint4 wraw[4 * JPW];
+        uint2 araw[JPW * NITG + 1];
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          wraw[c] = *reinterpret_cast<const uint4*>(pw + row * 128 + ((c ^ (row & 7)) << 4));
-        uint2 araw[NIT];
-        if constexpr (!AQ8) {
-          const uint8_t* pa = pw + C::PKW;
+        for (int jj = 0; jj < JPW; ++jj) {
+          const int j = cwg + C::CWG * jj;
+          if (j < nk) {
 #pragma unroll
-          for (int x = 0; x < NIT; ++x) {
-            // unit v = row pair index: rows r and r+4 of an 8-row block share a load
-            // phase, and their 16-byte chunks fall in different banks
-            const int it = ct + 128 * x;
-            const int j = it / (BT * 8), rem = it % (BT * 8);
-            const int v = rem >> 3, u = rem & 7;
-            const int r = (v & ~7) | ((v & 1) << 2) | ((v >> 1) & 3);
-            araw[x] = *reinterpret_cast<const uint2*>(
-                pa + r * 128 + (((4 * j + (u >> 1)) ^ (r & 7)) << 4) + ((u & 1) << 3));
+            for (int c = 0; c < 4; ++c)
+              wraw[4 * jj + c] = *reinterpret_cast<const uint4*>(
+                  pw + row * 128 + (((4 * j + c) ^ (row & 7)) << 4));
+            if constexpr (!AQ8) {
+              const uint8_t* pa = pw + C::PKW;
+#pragma unroll
+              for (int x = 0; x < NITG; ++x) {
+                // unit (v, u): token row v, 8-byte unit u of its 64 packed bytes.  Rows r
+                // and r+4 of an 8-row block share a load phase, so their 16-byte chunks
+                // fall in different banks.
+                const int it = ct + 128 * x;
+                const int v = it >> 3, u = it & 7;
+                const int r = (v & ~7) | ((v & 1) << 2) | ((v >> 1) & 3);
+                araw[jj * NITG + x] = *reinterpret_cast<const uint2*>(
+                    pa + r * 128 + (((4 * j + (u >> 1)) ^ (r & 7)) << 4) + ((u & 1) << 3));
+              }
+            }
           }
         }
 #pragma unroll
-        for (int j = 0; j < C::KPS; ++j) {
-          if (j < nk) {
-            const int xs = (i + j) % C::NX;
+        for (int jj = 0; jj < JPW; ++jj) {
+          const int j = cwg + C::CWG * jj;
+          if (j >= nk) continue;
+          const int xs = C::slot(q, i + j, j);
+          if constexpr (C::WSM) {
+            // the row's 128 expanded bytes, 16-byte chunk c at c ^ (row & 7)
+            uint8_t* wdst = xw + xs * C::XW + row * 128;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const uint4 a = wraw[4 * jj + cc];
+              *reinterpret_cast<uint4*>(wdst + (((2 * cc) ^ (row & 7)) << 4)) =
+                  make_uint4(expand_lo(a.x), expand_hi(a.x), expand_lo(a.y), expand_hi(a.y));
+              *reinterpret_cast<uint4*>(wdst + (((2 * cc + 1) ^ (row & 7)) << 4)) =
+                  make_uint4(expand_lo(a.z), expand_hi(a.z), expand_lo(a.w), expand_hi(a.w));
+            }
+          } else {
             uint32_t e0[16], e1[16];
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-              const uint4 a = wraw[4 * j + c], b = wraw[4 * j + 2 + c];
+              const uint4 a = wraw[4 * jj + c], b = wraw[4 * jj + 2 + c];
               e0[8 * c + 0] = expand_lo(a.x); e0[8 * c + 1] = expand_hi(a.x);
               e0[8 * c + 2] = expand_lo(a.y); e0[8 * c + 3] = expand_hi(a.y);
               e0[8 * c + 4] = expand_lo(a.z); e0[8 * c + 5] = expand_hi(a.z);
@@ -423,34 +531,39 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
             tmem_st16(tw, e0);
             tmem_st16(tw + 16, e1);
           }
-        }
-        if constexpr (!AQ8) {
+          if constexpr (!AQ8) {
 #pragma unroll
-          for (int x = 0; x < NIT; ++x) {
-            const int it = ct + 128 * x;
-            const int j = it / (BT * 8), rem = it % (BT * 8);
-            const int v = rem >> 3, u = rem & 7;
-            const int r = (v & ~7) | ((v & 1) << 2) | ((v >> 1) & 3);
-            if (j < nk) {
-              uint4 o;
-              o.x = expand_lo(araw[x].x);
-              o.y = expand_hi(araw[x].x);
-              o.z = expand_lo(araw[x].y);
-              o.w = expand_hi(araw[x].y);
-              *reinterpret_cast<uint4*>(xa + ((i + j) % C::NX) * C::XA + r * 128 +
-                                        ((u ^ (r & 7)) << 4)) = o;
+            for (int x = 0; x < NITG; ++x) {
+              const int it = ct + 128 * x;
+              const int v = it >> 3, u = it & 7;
+              const int r = (v & ~7) | ((v & 1) << 2) | ((v >> 1) & 3);
+              const uint2 w2 = araw[jj * NITG + x];
+              *reinterpret_cast<uint4*>(xa + xs * C::XA + r * 128 + ((u ^ (r & 7)) << 4)) =
+                  make_uint4(expand_lo(w2.x), expand_hi(w2.x), expand_lo(w2.y),
+                             expand_hi(w2.y));
             }
           }
-          fence_proxy_async_smem();
         }
-        tmem_st_wait();
-        tc_fence_before();
+        if constexpr (!AQ8) fence_proxy_async_smem();
+        if constexpr (!C::WSM) {
+          tmem_st_wait();
+          tc_fence_before();
+        }
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(smem_u32(&pk_empty[st]));
-          for (int j = 0; j < nk; ++j) mbar_arrive(smem_u32(&x_full[(i + j) % C::NX]));
+          if constexpr (C::GPB != 1) {
+            mbar_arrive(smem_u32(&x_full[q % C::NXU]));
+          } else {
+#pragma unroll
+            for (int jj = 0; jj < JPW; ++jj) {
+              const int j = cwg + C::CWG * jj;
+              if (j < nk) mbar_arrive(smem_u32(&x_full[(i + j) % C::NXU]));
+            }
+          }
         }
         if (lane == 0 && (warp & 3) == 2) trace_stamp(args, 1, q);
+        if (lane == 0) trace_stamp(args, 11 + (warp & 3), q);
         i += nk;
       }
     }
@@ -478,8 +591,11 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
     };
 
     float2 acc[C::CPT / 2];
+    // Narrow tiles pipeline the partial loads within a hand-off unit.
+    constexpr bool PIPE = C::CPT == 16 && C::GPB > 1;
     bool ok = true, aborted = false;
     int i = 0;     // flat group counter of this CTA
+    int u = 0;     // flat hand-off unit counter of this CTA
     int buf = 0;   // token-scale buffer in use
     Seg sg, nx;
     bool have = get_seg(args, 0, sg);
@@ -496,6 +612,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
 #pragma unroll
       for (int e = 0; e < C::CPT / 2; ++e) acc[e] = make_float2(0.0f, 0.0f);
       float sw_hoisted = 0.0f;
+      uint32_t pc[16];   // partials of the group in hand (units never straddle segments)
       for (int gb8 = sg.gb & ~7; gb8 < sg.ge; gb8 += 8) {
         // the next block's scales are in flight while this block is processed
         uint4 sa_n, sw_n;
@@ -516,20 +633,23 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
         const int jb = max(sg.gb - gb8, 0), je = min(sg.ge - gb8, 8);
 #pragma unroll 1
         for (int j = jb; j < je; ++j, ++i) {
-          const int sl = i % C::NSLOT;
-          ok = mbar_wait(smem_u32(&d_full[sl]), (uint32_t)(i / C::NSLOT) & 1u, lim, abort_flag);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          if (et == 0) trace_stamp(args, 7, i);
-          tc_fence_after();
+          const int r = (gb8 + j - sg.gb) % C::GPB;   // position in its hand-off unit
+          const bool unit_last = r == C::GPB - 1 || gb8 + j == sg.ge - 1;
+          const int sl = (u % C::NDU) * C::GPB + r;
+          if (r == 0) {
+            ok = mbar_wait(smem_u32(&g_done[u % C::NXU]), (uint32_t)(u / C::NXU) & 1u, lim,
+                           abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            if (et == 0) trace_stamp(args, 7, i);
+            tc_fence_after();
+          }
           const float4* sab = reinterpret_cast<const float4*>(sat + j * BT + h * 64);
           const float swj = half_of(sw_c, j) * (1.0f / 256.0f);
           const float2 sw2 = make_float2(swj, swj);
           const uint32_t td = tbase + t_lane + C::D_COL0 + sl * BT + h * 64;
-#pragma unroll
-          for (int cc = 0; cc < C::CPT / 16; ++cc) {
-            uint32_t p[16];
-            tmem_ld16(td + cc * 16, p);
+          // dequantise and accumulate 16 partials (columns cc*16 ..) of this group
+          auto consume = [&](const uint32_t* p, int cc) {
             if constexpr (DUMP) {
               const int g = gb8 + j;
 #pragma unroll
@@ -555,19 +675,44 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
                 acc[cc * 8 + 2 * qq + 1] = __ffma2_rn(pb, sa_b, acc[cc * 8 + 2 * qq + 1]);
               }
             }
+          };
+          if constexpr (PIPE) {
+            // the unit's first group is loaded here; every later one was loaded while the
+            // group before it was being processed
+            if (r == 0) {
+              tmem_ld16_nowait(td, pc);
+              tmem_ld_wait16(pc);
+            }
+            uint32_t pn[16];
+            if (!unit_last) tmem_ld16_nowait(td + BT, pn);
+            consume(pc, 0);
+            if (!unit_last) {
+              tmem_ld_wait16(pn);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) pc[e] = pn[e];
+            }
+          } else {
+#pragma unroll
+            for (int cc = 0; cc < C::CPT / 16; ++cc) {
+              uint32_t p[16];
+              tmem_ld16(td + cc * 16, p);
+              consume(p, cc);
+            }
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(smem_u32(&d_empty[sl]));
-            if (et == 0) trace_stamp(args, 3, i);
+          if (unit_last) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&d_empty[u % C::NDU]));
+            ++u;
           }
+          if (et == 0) trace_stamp(args, 3, i);
         }
         buf ^= 1;
         sa_c = sa_n;
         sw_c = sw_n;
       }
       // ---- segment finished: write the tile, or hand its partial to the fixup
+      if (et == 0) trace_stamp(args, 15, 4 * k);
       aborted = aborted || bar_red_or(1, NE, !ok);
       if (aborted) break;
       if constexpr (!DUMP) {
@@ -576,9 +721,8 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
 #pragma unroll
           for (int e = 0; e < C::CPT / 2; ++e) acc[e] = __fmul2_rn(acc[e], sh);
         }
-        const long long tu0 = (long long)sg.t * args.S;
-        const int cf = args.streamk ? sk_owner(args, tu0) : (int)blockIdx.x;
-        const int cl = args.streamk ? sk_owner(args, tu0 + args.S - 1) : (int)blockIdx.x;
+        const int cf = args.streamk ? sk_owner(args, sg.t * args.S) : (int)blockIdx.x;
+        const int cl = args.streamk ? sk_owner(args, sg.t * args.S + args.S - 1) : (int)blockIdx.x;
         if (cf == cl) {
 #pragma unroll
           for (int e = 0; e < C::CPT; ++e) {
@@ -590,7 +734,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
           // partial slot: 0 for this CTA's first tile, 1 for its last (a CTA shares at most
           // those two tiles with other CTAs)
           auto slot_of = [&](int c) -> size_t {
-            const int tf = (int)(sk_u0(args, c) / args.S);
+            const int tf = sk_u0(args, c) / args.S;
             return ((size_t)c * 2 + (sg.t == tf ? 0 : 1)) * (size_t)(BT * C::BM);
           };
           float* mine = args.part + slot_of(blockIdx.x);
@@ -599,29 +743,43 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
             const int ml = h * 64 + e;
             mine[(size_t)ml * C::BM + row] = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
           }
-          __threadfence();
+          // publish: the barrier collects every thread's stores, one thread releases them
+          // with the arrival; the last arrival acquires everyone's before the sum
           bar_red_or(1, NE, false);
+          if (et == 0) trace_stamp(args, 15, 4 * k + 1);
           if (et == 0) {
+            fence_acq_rel_gpu();
             const unsigned old = atomicAdd(&args.counters[sg.t], 1u);
-            *reinterpret_cast<volatile int*>(s_last) = (old == (unsigned)(cl - cf));
+            const int last = old == (unsigned)(cl - cf);
+            if (last) fence_acq_rel_gpu();
+            *reinterpret_cast<volatile int*>(s_last) = last;
           }
           bar_red_or(1, NE, false);
+          if (et == 0) trace_stamp(args, 15, 4 * k + 2);
           if (*reinterpret_cast<volatile int*>(s_last)) {
-            __threadfence();
-            // the contributions, added in CTA order whoever arrives last
+            // the contributions, added in CTA order whoever arrives last; NCH CTAs' values
+            // are in flight at once
+            constexpr int NCH = 2;
 #pragma unroll
             for (int e0 = 0; e0 < C::CPT; e0 += 16) {
               float sum[16];
 #pragma unroll
               for (int e = 0; e < 16; ++e) sum[e] = 0.0f;
-              for (int c = cf; c <= cl; ++c) {
-                const float* src = args.part + slot_of(c);
-                float v[16];
+              for (int c = cf; c <= cl; c += NCH) {
+                float v[NCH][16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                  v[e] = __ldcg(src + (size_t)(h * 64 + e0 + e) * C::BM + row);
+                for (int cc = 0; cc < NCH; ++cc) {
+                  const float* src = args.part + slot_of(min(c + cc, cl));
 #pragma unroll
-                for (int e = 0; e < 16; ++e) sum[e] += v[e];
+                  for (int e = 0; e < 16; ++e)
+                    v[cc][e] = c + cc <= cl
+                                   ? __ldcg(src + (size_t)(h * 64 + e0 + e) * C::BM + row)
+                                   : 0.0f;
+                }
+#pragma unroll
+                for (int cc = 0; cc < NCH; ++cc)
+#pragma unroll
+                  for (int e = 0; e < 16; ++e) sum[e] += v[cc][e];
               }
 #pragma unroll
               for (int e = 0; e < 16; ++e) {
@@ -633,6 +791,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
           }
         }
       }
+      if (et == 0) trace_stamp(args, 15, 4 * k + 3);
       have = have_next;
       sg = nx;
     }

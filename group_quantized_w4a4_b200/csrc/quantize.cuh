@@ -18,6 +18,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include "ptx.cuh"
+
 namespace apex {
 
 __device__ __forceinline__ float absmax8(const uint4& v) {
@@ -63,6 +65,10 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __rest
                                                             int64_t rows, int64_t K, int group,
                                                             uint8_t* __restrict__ packed,
                                                             __half* __restrict__ scales) {
+  // launched as a programmatic dependent: nothing is read or written before the previous
+  // grid in the stream has completed
+  grid_dep_wait();
+  grid_dep_launch();
   const int64_t G = K / group;
   const int64_t units = rows * G;
   const int chunks = group / 128;

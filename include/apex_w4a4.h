@@ -164,15 +164,18 @@ void apex_debug_withhold_step(int32_t step);
 
 /*
  * Tracing hook: the next apex_w4a4_gemm launch on this host thread writes timestamps for
- * its first `ctas` CTAs (persistent CTA index) into the device buffer trace[ctas][10][steps]
+ * its first `ctas` CTAs (persistent CTA index) into the device buffer trace[ctas][16][steps]
  * (uint64).  SM clock cycles (clock64): [c][0][s] producer issued stage s (a pair of
  * K-groups), [c][1][s] converters done with stage s, [c][2][i] MMAs of K-group i issued,
  * [c][3][i] epilogue done with K-group i, [c][4][s] converter inputs of stage s ready,
  * [c][6][i] MMA inputs of K-group i ready (after the tensor-core fence), [c][7][i]
  * epilogue inputs of K-group i ready, [c][8][i] MMA waits returned, [c][9][i] MMAs of
- * K-group i issued before their commits;
+ * K-group i issued before their commits, [c][10][i] MMA wait for the operands of K-group i
+ * returned, [c][11 + w][s] converter warp w (0..3 within its warpgroup) done with stage s;
  * [c][5][0] / [c][5][1] %globaltimer (ns) at CTA start / end, [c][5][2] the SM it ran on,
- * [c][5][3] clock64 at CTA start.  Steps beyond `steps` are not recorded.
+ * [c][5][3] clock64 at CTA start, [c][5][4] / [c][5][5] clock64 when the producer enters its
+ * loop / has its first work item, [c][5][6] %globaltimer at kernel entry (before the
+ * prologue).  Steps beyond `steps` are not recorded.
  */
 void apex_debug_trace_next_gemm(uint64_t *trace, int32_t ctas, int32_t steps);
 
