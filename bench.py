@@ -285,10 +285,11 @@ def e2e_workload(apex, torch, g, steps, warmup, p: Problem):
 def roofline_obj(g, gemm_ms_avg, peaks, peaks_kind, traffic=None):
     hbm = float(peaks["hbm_gbs"]) * 1e9
     i8 = float(peaks.get("bf16_tflops", 1590.0)) * 1e12 * INT8_PER_BF16
-    t_bound, bound = roofline.bound_time_s(g.ops, g.gemm_bytes(), i8, hbm)
+    nbytes = g.gemm_bytes(g.M >= EXPANDED_MIN_M)
+    t_bound, bound = roofline.bound_time_s(g.ops, nbytes, i8, hbm)
     t = gemm_ms_avg * 1e-3
     if bound == "hbm":
-        achieved = g.gemm_bytes() / t / 1e9
+        achieved = nbytes / t / 1e9
         peak = float(peaks["hbm_gbs"])
         unit = "GB/s"
         note = f"hbm_gbs of {peaks_kind}"
@@ -300,7 +301,7 @@ def roofline_obj(g, gemm_ms_avg, peaks, peaks_kind, traffic=None):
     return {"bound": "hbm" if bound == "hbm" else "tensor", "achieved": round(achieved, 2),
             "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
             "traffic": traffic, "peak_source": note,
-            "algorithmic_bytes": g.gemm_bytes(), "ops": g.ops,
+            "algorithmic_bytes": nbytes, "ops": g.ops,
             "kernel_ms": round(gemm_ms_avg, 5)}
 
 
@@ -366,6 +367,7 @@ def run_apex(args, rank, world, local):
         del p2
     if rank != 0:
         return None
+    expd = g.M >= EXPANDED_MIN_M
     line = {
         "metric": "W4A4-g128 GEMM effective TOPS (quantize + GEMM step) and % of roofline",
         "value": round(value, 2), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
@@ -384,9 +386,9 @@ def run_apex(args, rank, world, local):
         "launch": ("one CUDA graph of the K timed steps (eager warm-up), kernels launched as "
                    "programmatic dependents; per-kernel times from two more graphs of K "
                    "launches of that kernel alone"),
-        "gemm": {"kernel_ms": round(gemm_avg, 5), "bytes": g.gemm_bytes()},
-        "quantize": {"kernel_ms": round(quant_avg, 5), "bytes": g.quant_bytes(),
-                     "GB/s": round(g.quant_bytes() / (quant_avg * 1e-3) / 1e9, 1)},
+        "gemm": {"kernel_ms": round(gemm_avg, 5), "bytes": g.gemm_bytes(expd)},
+        "quantize": {"kernel_ms": round(quant_avg, 5), "bytes": g.quant_bytes(expd),
+                     "GB/s": round(g.quant_bytes(expd) / (quant_avg * 1e-3) / 1e9, 1)},
         "clocks": clk,
         "impl": "apex",
     }
@@ -395,6 +397,37 @@ def run_apex(args, rank, world, local):
     if world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(g)
     return line
+
+
+def run_sweep(args, rank, world, local):
+    """One JSON line per secondary workload: the mixed-granularity sweep (M x weight group)
+    and the MLP pair, each timed like the headline (step, GEMM alone, quantizer alone)."""
+    import torch
+    import group_quantized_w4a4_b200 as apex
+    apex.load_library()
+    torch.cuda.set_device(local)
+    props = torch.cuda.get_device_properties(local)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 1024 * 1024))
+    peaks, peaks_kind = load_peaks()
+    names = [n for n in synth.workloads() if n.startswith("sweep_") or n.startswith("mlp_")]
+    steps = max(3, args.steps // 4)
+    lines = []
+    for name in names:
+        g = synth.workloads()[name]
+        p, tot, gm, _, qm = time_workload(apex, torch, g, steps, args.warmup, world, l2)
+        del p
+        torch.cuda.empty_cache()
+        ms = max_over_ranks(tot / steps, world)
+        gm, qm = max_over_ranks(gm, world), max_over_ranks(qm, world)
+        lines.append({
+            "sweep": name, "M": g.M, "N": g.N, "K": g.K, "group_a": 128, "group_w": g.gw,
+            "steps": steps, "activation_form": "expanded" if g.M >= EXPANDED_MIN_M else "packed",
+            "step_ms": round(ms, 5), "gemm_ms": round(gm, 5), "quantize_ms": round(qm, 5),
+            "step_TOPS": round(world * g.ops / (ms * 1e-3) / 1e12, 2),
+            "gemm_TOPS": round(g.ops / (gm * 1e-3) / 1e12, 2),
+            "gemm_GBs": round(g.gemm_bytes(g.M >= EXPANDED_MIN_M) / (gm * 1e-3) / 1e9, 1),
+            "roofline": roofline_obj(g, gm, peaks, peaks_kind)})
+    return lines if rank == 0 else None
 
 
 def p_copies(g, l2):
@@ -434,17 +467,23 @@ def main():
     ap.add_argument("--impl", default="apex", choices=["apex", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     ap.add_argument("--no-second", action="store_true", help="skip the M=4096 companion line")
+    ap.add_argument("--sweep", action="store_true",
+                    help="instead of the headline line, one line per sweep / MLP workload")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank, world, local = dist_init(args.gpus)
     try:
-        if args.impl == "reference":
-            line = run_reference(args, rank, world)
+        if args.sweep:
+            for line in run_sweep(args, rank, world, local) or []:
+                print(json.dumps(line), flush=True)
         else:
-            line = run_apex(args, rank, world, local)
-        if line is not None:
-            print(json.dumps(line), flush=True)
+            if args.impl == "reference":
+                line = run_reference(args, rank, world)
+            else:
+                line = run_apex(args, rank, world, local)
+            if line is not None:
+                print(json.dumps(line), flush=True)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -79,16 +79,18 @@ class Gemm:
     def ops(self) -> float:
         return 2.0 * self.M * self.N * self.K
 
-    def gemm_bytes(self) -> int:
-        """Algorithmic HBM bytes of one GEMM call: packed A and W, fp16 scales, fp16 Y."""
+    def gemm_bytes(self, expanded: bool = False) -> int:
+        """Algorithmic HBM bytes of one GEMM call: A (packed, or one byte per element in the
+        expanded form) and packed W, fp16 scales, fp16 Y."""
         M, N, K = self.M, self.N, self.K
-        return (M * K // 2 + N * K // 2 + 2 * M * (K // self.ga)
+        a = M * K if expanded else M * K // 2
+        return (a + N * K // 2 + 2 * M * (K // self.ga)
                 + 2 * N * (K // self.gw) + 2 * M * N)
 
-    def quant_bytes(self) -> int:
+    def quant_bytes(self, expanded: bool = False) -> int:
         """Algorithmic HBM bytes of the online activation quantizer."""
         M, K = self.M, self.K
-        return 2 * M * K + M * K // 2 + 2 * M * (K // self.ga)
+        return 2 * M * K + (M * K if expanded else M * K // 2) + 2 * M * (K // self.ga)
 
 
 def workloads() -> dict:

@@ -171,7 +171,9 @@ void apex_debug_withhold_step(int32_t step);
  * [c][6][i] MMA inputs of K-group i ready (after the tensor-core fence), [c][7][i]
  * epilogue inputs of K-group i ready, [c][8][i] MMA waits returned, [c][9][i] MMAs of
  * K-group i issued before their commits, [c][10][i] MMA wait for the operands of K-group i
- * returned, [c][11 + w][s] converter warp w (0..3 within its warpgroup) done with stage s;
+ * returned, [c][11 + w][s] converter warp w (0..3 within its warpgroup) done with stage s,
+ * [c][15][4k .. 4k+3] the epilogue's k-th segment: finished, partial published, arrival
+ * counted, tile written;
  * [c][5][0] / [c][5][1] %globaltimer (ns) at CTA start / end, [c][5][2] the SM it ran on,
  * [c][5][3] clock64 at CTA start, [c][5][4] / [c][5][5] clock64 when the producer enters its
  * loop / has its first work item, [c][5][6] %globaltimer at kernel entry (before the
