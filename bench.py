@@ -15,6 +15,8 @@ an independent replica (the path has no exchange step), time = max over ranks.
 from __future__ import annotations
 
 import argparse
+import glob
+import hashlib
 import json
 import os
 import statistics
@@ -282,6 +284,30 @@ def e2e_workload(apex, torch, g, steps, warmup, p: Problem):
     return ms, x_host.numel() * 2, y_host.numel() * 2
 
 
+def kernel_source_hash() -> str:
+    """sha256 (first 16 hex) of the CUDA sources, to tell whether recorded counters still
+    describe the kernel that runs."""
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "group_quantized_w4a4_b200", "csrc", "*"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(name: str):
+    """DRAM bytes per GEMM launch from the last ncu capture of this workload, or None when
+    there is none or the kernel sources changed since it was taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
+            rec = json.load(fh)
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("traffic_bytes_per_launch", {}).get(name)
+
+
 def roofline_obj(g, gemm_ms_avg, peaks, peaks_kind, traffic=None):
     hbm = float(peaks["hbm_gbs"]) * 1e9
     i8 = float(peaks.get("bf16_tflops", 1590.0)) * 1e12 * INT8_PER_BF16
@@ -300,7 +326,8 @@ def roofline_obj(g, gemm_ms_avg, peaks, peaks_kind, traffic=None):
         note = f"int8 = {INT8_PER_BF16:g} x bf16_tflops of {peaks_kind} (nominal int8:bf16 ratio)"
     return {"bound": "hbm" if bound == "hbm" else "tensor", "achieved": round(achieved, 2),
             "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
-            "traffic": traffic, "peak_source": note,
+            "traffic": traffic if traffic is not None else recorded_traffic(g.name),
+            "peak_source": note,
             "algorithmic_bytes": nbytes, "ops": g.ops,
             "kernel_ms": round(gemm_ms_avg, 5)}
 
