@@ -134,7 +134,8 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, bool allow_streamk) {
   p.tiles_m = (int)((M + p.bt - 1) / p.bt);
   p.T = p.tiles_n * p.tiles_m;
   const int G = (int)(K / 128);
-  p.S = (G + 1) / 2;
+  const int kps = apex::stage_groups(p.bt);
+  p.S = (G + kps - 1) / kps;
   const int sms = dev_info().sms;
   if (!allow_streamk || p.T >= 4 * sms) {
     p.streamk = 0;
@@ -142,7 +143,12 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, bool allow_streamk) {
   } else {
     p.streamk = 1;
     const long long units = (long long)p.T * p.S;
-    p.P = units < sms ? (int)units : sms;
+    // With at least two CTAs per tile, split every tile the same number of ways: each CTA
+    // then holds one piece of one tile and finishes with a single hand-off, instead of
+    // stream-K's pieces of two tiles (a few SMs idle, but the split-K tail halves).
+    const int per_tile = sms / p.T;
+    const long long want = per_tile >= 2 ? (long long)per_tile * p.T : sms;
+    p.P = units < want ? (int)units : (int)want;
     if ((long long)p.P * units >= (1ll << 31)) {   // the device partition math is 32-bit
       p.streamk = 0;
       p.P = p.T < sms ? p.T : sms;
@@ -155,7 +161,7 @@ size_t counters_bytes(const Plan& p) { return (((size_t)p.T * 4) + 255) & ~(size
 
 size_t workspace_for(const Plan& p) {
   if (!p.streamk) return 0;
-  return counters_bytes(p) + (size_t)p.P * 2 * (size_t)p.bt * 128 * 4;
+  return counters_bytes(p) + (size_t)p.P * (size_t)p.bt * 128 * 4;
 }
 
 apex_status_t check_gemm_args(int64_t M, int64_t N, int64_t K, int32_t ga, int32_t gw) {
@@ -227,10 +233,15 @@ GemmArgs base_args(const Plan& p, int64_t M, int64_t N, int64_t K, int32_t gw,
   a.gw = gw;
   a.G = (int)(K / 128);
   a.Gw = (int)(K / gw);
+  {
+    const int gpg = gw / 128;
+    a.gpg_shift = (gpg & (gpg - 1)) == 0 ? __builtin_ctz((unsigned)gpg) : -1;
+  }
   a.tiles_n = p.tiles_n;
   a.tiles_m = p.tiles_m;
   a.T = p.T;
   a.S = p.S;
+  a.kps = apex::stage_groups(p.bt);
   a.TS = p.streamk ? p.T * p.S : 0;
   a.P = p.P;
   a.streamk = p.streamk;

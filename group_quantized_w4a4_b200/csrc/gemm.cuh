@@ -15,19 +15,18 @@
 //   tile mode     whole tiles, round-robin over the CTAs (many tiles);
 //   stream-K      the tiles' K-stages are cut into equal contiguous ranges, one per CTA, so
 //                 every SM streams the same number of bytes (few tiles: decode, small M).
-//                 A tile covered by several CTAs is finished by the last one to arrive,
-//                 which adds the fp32 partials in CTA order (deterministic).
+//                 A tile covered by several CTAs is finished by the CTA holding its first
+//                 stage, which adds the others' fp32 parts in CTA order (deterministic).
 // Roles:
-//   warp 0      TMA producer: packed W tile [128 x 128 B] (two K-groups per stage) and
+//   warp 0      TMA producer: packed W tile, one [128 x 128 B] box per two K-groups (a stage
+//               holds two K-groups, four for tiles of at most 32 tokens), and
 //               the token tile -- packed [BT x 128 B], or, in the expanded-activation mode,
 //               one [BT x 128 B] int8 tile per group straight into the MMA operand slot.
 //   warp 1      MMA issuer (one thread): 4 x tcgen05.mma kind::i8 (K = 32 each) per group
 //               into a tensor-memory slot; one exact int32 partial per group.
-//   warps 2..   converters (one warpgroup; for narrow tiles two, each taking one of the
-//               two K-groups of every stage): nibbles -> int8 in registers.  The weight row
-//               of each thread goes to tensor memory (tcgen05.st) for wide tiles, or to
-//               shared memory for narrow ones; packed token rows go to shared memory.  Both
-//               shared-memory operands use the 128-byte-swizzled K-major layout.
+//   warps 2..5  converters (one warpgroup): nibbles -> int8 in registers.  The weight row
+//               of each thread goes to tensor memory (tcgen05.st); packed token rows go to
+//               shared memory in the 128-byte-swizzled K-major operand layout.
 //   then        epilogue: tcgen05.ld of a group's partials while the next groups' MMAs
 //               run, fp32 scale by sa*sw and accumulate in registers (packed f32x2 math);
 //               fp16 output.  Each epilogue thread also fetches the scales it needs, one
@@ -56,10 +55,12 @@ enum GemmMode : int { MODE_PACKED = 0, MODE_AQ8 = 1, MODE_DUMP = 2 };
 struct GemmArgs {
   int M, N, K;
   int gw;            // weight group (multiple of 128 dividing K)
+  int gpg_shift;     // log2(gw / 128) when that is a power of two, else -1
   int G;             // K / 128
   int Gw;            // K / gw
   int tiles_n, tiles_m, T;   // tiles (n fastest)
-  int S;             // K-stages (pairs of groups) per tile
+  int S;             // K-stages per tile
+  int kps;           // K-groups per stage (stage_groups(BT))
   int TS;            // T * S
   int P;             // persistent CTAs (gridDim.x)
   int streamk;       // 1: contiguous stage ranges per CTA; 0: whole tiles round-robin
@@ -68,14 +69,14 @@ struct GemmArgs {
   const __half* sa;  // [M][G]
   const __half* sw;  // [N][Gw]
   __half* y;         // [M][N]
-  float* part;       // stream-K partial tiles [P][2][BT][128] fp32
+  float* part;       // stream-K partial tiles [P][BT][128] fp32 (one per CTA)
   unsigned* counters;  // [T] arrival counters of split tiles (zero between calls)
   int32_t* dump;     // [G][M][N] per-group partials (debug kernel only)
   unsigned long long wait_ns;
   int withhold;      // test hook: the producer never loads this stage (-1: off)
   // Optional timeline trace (null: off), for the first trace_ctas CTAs:
   // SM clock stamps (clock64) [cta][role][step] with roles 0 producer issue, 1 converter
-  // done and 4 converter inputs ready (per stage of two K-groups), 2 MMA issued, 3
+  // done and 4 converter inputs ready (per stage), 2 MMA issued, 3
   // epilogue done, 6 MMA inputs ready, 7 epilogue inputs ready, 8 MMA waits returned and
   // 9 MMAs issued before their commits (per K-group);
   // [cta][5][0..1] = %globaltimer at start / end, [cta][5][2] = the SM the CTA ran on,
@@ -103,6 +104,10 @@ __device__ __forceinline__ void trace_stamp(const GemmArgs& a, int role, int ste
       role == 5 ? globaltimer_ns() : clock_cycles();
 }
 
+// K-groups per pipeline stage: narrow tiles move four groups per stage (two 128-byte TMA
+// boxes of packed weights), so the per-stage hand-off costs are spread over more MMAs.
+__host__ __device__ constexpr int stage_groups(int bt) { return bt <= 32 ? 4 : 2; }
+
 #ifndef APEX_WSM_MAX_BT
 #define APEX_WSM_MAX_BT 0
 #endif
@@ -114,13 +119,18 @@ struct GemmCfg {
   // shared memory); wide tiles keep it in tensor memory.
   static constexpr bool WSM = !AQ8 && BT <= APEX_WSM_MAX_BT;
   static constexpr int BM = 128;
-  static constexpr int KPS = 2;                                    // K-groups per packed stage
+  static constexpr int KPS = stage_groups(BT);                     // K-groups per packed stage
+  static constexpr int NBOX = KPS / 2;                             // 128-byte boxes per stage
   // operand slots (per group): expanded weight tile (tensor or shared memory) + token tile
   static constexpr int NX = WSM ? (BT <= 32 ? 6 : 4) : BT >= 128 ? (AQ8 ? 6 : 4) : 8;
-  static constexpr int NSLOT = WSM ? NX : BT >= 128 ? (AQ8 ? 2 : 3) : 4;  // partial (D) slots
-  static constexpr int EPI_WARPS = BT >= 128 ? 8 : 4;
+  static constexpr int NSLOT = WSM ? NX : BT >= 128 ? (AQ8 ? 2 : 3) : KPS == 4 ? 8 : 4;
+  // Epilogue: 8 warps.  Wide tiles split the 128 columns in two halves; narrow tiles run
+  // two teams of 4 warps that take alternate hand-off units (so one team's TMEM loads and
+  // waits overlap the other's arithmetic) and add their sums at the end of a segment.
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int TEAMS = BT >= 128 ? 1 : 2;
   static constexpr int CPT = BT >= 128 ? 64 : BT;  // columns per epilogue thread
-  static constexpr int CWG = BT >= 128 ? 1 : 2;    // converter warpgroups (alternate stages)
+  static constexpr int CWG = 1;                    // converter warpgroups
   static constexpr int CONV0 = 2;                  // first converter warp
   static constexpr int EPI0 = CONV0 + 4 * CWG;     // first epilogue warp
   static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
@@ -135,14 +145,16 @@ struct GemmCfg {
   static constexpr int XA = BT * 128;                    // one group's int8 token tile
   static constexpr int XW = WSM ? BM * 128 : 0;          // one group's int8 weight tile
   static constexpr int SAT = 2 * 8 * BT * 4;  // token scales: 2 blocks x [8 groups][BT] fp32
-  static constexpr int FIXED = NX * (XA + XW) + SAT + 4096;
+  static constexpr int RED = TEAMS == 2 ? CPT * BM * 4 : 0;   // second team's sums [CPT][BM]
+  static constexpr int FIXED = NX * (XA + XW) + SAT + RED + 4096;
   static constexpr int NP_FIT = (200 * 1024 - FIXED) / PK_STAGE;
   static constexpr int NP = NP_FIT > 12 ? 12 : (NP_FIT < 2 ? 2 : NP_FIT);  // packed stages
   static constexpr int OFF_PK = 0;
   static constexpr int OFF_XA = OFF_PK + NP * PK_STAGE;
   static constexpr int OFF_XW = OFF_XA + NX * XA;
   static constexpr int OFF_SAT = OFF_XW + NX * XW;
-  static constexpr int OFF_BAR = OFF_SAT + SAT;
+  static constexpr int OFF_RED = OFF_SAT + SAT;
+  static constexpr int OFF_BAR = OFF_RED + RED;
   // Hand-off unit: the groups that pass between converters, MMA and epilogue under one
   // barrier phase -- a whole stage for narrow tiles (the MMA issue loop is short on work
   // per group there), a single group for wide ones (whose partial slots fill TMEM).
@@ -171,16 +183,38 @@ __device__ __forceinline__ uint32_t expand_hi(uint32_t w) { return w & 0xF0F0F0F
 
 // The 8 fp16 scales of groups gbeg .. gbeg+7 of one row, as raw bits (zeros outside
 // [glo, ghi)).  vec: one 16-byte load (gbeg a multiple of 8, 16-byte aligned rows, weight
-// group == 128).  Otherwise element loads of base[row_off + g*128/gw].
+// group == 128).  Otherwise the scale of group g is base[row_off + g / gpg] (gpg = K-groups
+// per scale group, gpg_shift = log2(gpg) when it is a power of two, else -1); when a scale
+// group covers 8 groups or more, each distinct scale of the block is loaded once.
 __device__ __forceinline__ uint4 load_scale_block(const __half* base, size_t row_off, int gbeg,
-                                                  int glo, int ghi, bool vec, int gw) {
+                                                  int glo, int ghi, bool vec, int gpg,
+                                                  int gpg_shift) {
   if (vec) return __ldg(reinterpret_cast<const uint4*>(base + row_off + gbeg));
+  const int lo = max(gbeg, glo), hi = min(gbeg + 8, ghi);   // groups of the block in use
   uint32_t h[8];
+  if (gpg >= 8 || lo >= hi) {
+    // at most two scale groups meet the block
+    const int s0 = lo / gpg, s1 = (hi - 1) / gpg;
+    const uint32_t v0 = lo < hi ? __half_as_ushort(base[row_off + s0]) : 0u;
+    const uint32_t v1 = (lo < hi && s1 != s0) ? __half_as_ushort(base[row_off + s1]) : v0;
+    const int split = (s0 + 1) * gpg;   // first group of the second scale group
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int g = gbeg + j;
-    h[j] = (g >= glo && g < ghi) ? __half_as_ushort(base[row_off + (size_t)((g * 128) / gw)])
-                                 : 0u;
+    for (int j = 0; j < 8; ++j) {
+      const int g = gbeg + j;
+      h[j] = (g >= lo && g < hi) ? (g < split ? v0 : v1) : 0u;
+    }
+  } else if (gpg_shift >= 0) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int g = gbeg + j;
+      h[j] = (g >= lo && g < hi) ? __half_as_ushort(base[row_off + (g >> gpg_shift)]) : 0u;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int g = gbeg + j;
+      h[j] = (g >= lo && g < hi) ? __half_as_ushort(base[row_off + g / gpg]) : 0u;
+    }
   }
   return make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
                     h[6] | (h[7] << 16));
@@ -229,8 +263,8 @@ __device__ __forceinline__ bool get_seg(const GemmArgs& a, int k, Seg& sg) {
   const int sb = t == tf ? u0 - tf * a.S : 0;
   const int se = t == tl ? (u1 - 1) - tl * a.S + 1 : a.S;
   sg.t = t;
-  sg.gb = sb * 2;
-  sg.ge = min(se * 2, a.G);
+  sg.gb = sb * a.kps;
+  sg.ge = min(se * a.kps, a.G);
   return true;
 }
 
@@ -248,6 +282,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
   uint8_t* xa = smem + C::OFF_XA;
   uint8_t* xw = smem + C::OFF_XW;
   float* s_sat = reinterpret_cast<float*>(smem + C::OFF_SAT);
+  float* s_red = reinterpret_cast<float*>(smem + C::OFF_RED);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* pk_full = bars;
   uint64_t* pk_empty = pk_full + C::NP;
@@ -272,15 +307,15 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NP; ++i) {
       mbar_init(smem_u32(&pk_full[i]), 1);
-      mbar_init(smem_u32(&pk_empty[i]), 4 * C::CWG);  // one arrival per converter warp
+      mbar_init(smem_u32(&pk_empty[i]), 1);   // one elected converter arrival
     }
     for (int i = 0; i < C::NXU; ++i) {
-      // one arrival per converter warp that fills the unit
-      mbar_init(smem_u32(&x_full[i]), C::GPB == 1 ? 4 : 4 * C::CWG);
+      mbar_init(smem_u32(&x_full[i]), 1);     // one elected converter arrival
       mbar_init(smem_u32(&g_done[i]), 1);
     }
     for (int i = 0; i < C::NDU; ++i) {
-      mbar_init(smem_u32(&d_empty[i]), C::EPI_WARPS);  // one arrival per epilogue warp
+      // one arrival per epilogue warp (one elected arrival per team for whole-stage units)
+      mbar_init(smem_u32(&d_empty[i]), C::GPB == 1 ? C::EPI_WARPS : 1);
     }
     mbar_init(smem_u32(mma_done), 1);
     *s_abort = 0;
@@ -351,14 +386,19 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
         }
         if (lane == 0) {
           const uint32_t fb = smem_u32(&pk_full[st]);
-          mbar_arrive_expect_tx(fb, C::PKW + (AQ8 ? nk * C::XA : C::PKA));
-          tma_load_2d(smem_u32(pk + st * C::PK_STAGE), &tmW, fb, g * 64, n0);
+          const int nb = (nk + 1) >> 1;   // 128-byte boxes that hold the stage's groups
+          mbar_arrive_expect_tx(fb, nb * (C::BM * 128) + (AQ8 ? nk * C::XA : nb * BT * 128));
+          for (int b = 0; b < nb; ++b)
+            tma_load_2d(smem_u32(pk + st * C::PK_STAGE + b * (C::BM * 128)), &tmW, fb,
+                        (g + 2 * b) * 64, n0);
           if constexpr (AQ8) {
             for (int j = 0; j < nk; ++j)
               tma_load_2d(smem_u32(xa + C::slot(q, i + j, j) * C::XA), &tmA, fb, (g + j) * 128,
                           m0);
           } else {
-            tma_load_2d(smem_u32(pk + st * C::PK_STAGE + C::PKW), &tmA, fb, g * 64, m0);
+            for (int b = 0; b < nb; ++b)
+              tma_load_2d(smem_u32(pk + st * C::PK_STAGE + C::PKW + b * (BT * 128)), &tmA, fb,
+                          (g + 2 * b) * 64, m0);
           }
           trace_stamp(args, 0, q);
         }
@@ -444,33 +484,32 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
       for (int g = sg.gb; g < sg.ge; g += C::KPS, ++q) {
         const int st = q % C::NP;
         const int nk = min(C::KPS, sg.ge - g);
-        // the stage's bytes, and the operand slots it fills.  With whole-stage units every
-        // converter warp waits for the unit's previous use (even a warpgroup with no group
-        // in a short stage), so its arrival can only count toward this use.
+        // The stage's bytes, and the operand slots it fills (their previous use done).  One
+        // warp waits; the others park in the hardware barrier below, where barrier events
+        // do not wake them.
         const uint32_t pf_par = (uint32_t)(q / C::NP) & 1u;
-        if constexpr (C::GPB != 1) {
-          ok = mbar_wait2(smem_u32(&pk_full[st]), pf_par, smem_u32(&g_done[q % C::NXU]),
-                          ((uint32_t)(q / C::NXU) & 1u) ^ 1u, lim, abort_flag);
-        } else {
-          ok = cwg < nk ? mbar_wait2(smem_u32(&pk_full[st]), pf_par,
-                                     smem_u32(&g_done[(i + cwg) % C::NXU]),
-                                     ((uint32_t)((i + cwg) / C::NXU) & 1u) ^ 1u, lim, abort_flag)
-                        : mbar_wait(smem_u32(&pk_full[st]), pf_par, lim, abort_flag);
-#pragma unroll
-          for (int jj = 1; jj < JPW; ++jj) {
-            const int j = cwg + C::CWG * jj;
-            if (j < nk)
+        if (ct < 32) {
+          if constexpr (C::GPB != 1) {
+            ok = mbar_wait2(smem_u32(&pk_full[st]), pf_par, smem_u32(&g_done[q % C::NXU]),
+                            ((uint32_t)(q / C::NXU) & 1u) ^ 1u, lim, abort_flag);
+          } else {
+            ok = mbar_wait2(smem_u32(&pk_full[st]), pf_par, smem_u32(&g_done[i % C::NXU]),
+                            ((uint32_t)(i / C::NXU) & 1u) ^ 1u, lim, abort_flag);
+            for (int j = 1; j < nk; ++j)
               ok = ok && mbar_wait(smem_u32(&g_done[(i + j) % C::NXU]),
                                    ((uint32_t)((i + j) / C::NXU) & 1u) ^ 1u, lim, abort_flag);
           }
         }
-        ok = __all_sync(0xffffffffu, ok);
+        // one decision for the whole warpgroup, so none of it can be left at the barrier
+        // below when another part gives up
+        ok = !bar_red_or(2, 128, !ok);
+        tc_fence_after();   // tensor-memory writes below come after the slots' last reads
         if (!ok) break;
         if (lane == 0 && (warp & 3) == 2) trace_stamp(args, 4, q);
         const uint8_t* pw = pk + st * C::PK_STAGE;
-        // All shared-memory reads first, so their latencies overlap.  Packed W row: the
-        // 16-byte chunk c of the 128-byte stage row sits at c ^ (row & 7); group j owns
-        // chunks 4j .. 4j+3.
+        // All shared-memory reads first, so their latencies overlap.  Packed W: group j of
+        // the stage lies in 128-byte box j / 2, chunks 4 (j % 2) .. +3 of the row, with the
+        // 16-byte chunk c of a box row stored at c ^ (row & 7).
         uint4 wraw[4 * JPW];
         uint2 araw[JPW * NITG + 1];
 #pragma unroll
@@ -480,7 +519,8 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c)
               wraw[4 * jj + c] = *reinterpret_cast<const uint4*>(
-                  pw + row * 128 + (((4 * j + c) ^ (row & 7)) << 4));
+                  pw + (j >> 1) * (C::BM * 128) + row * 128 +
+                  (((4 * (j & 1) + c) ^ (row & 7)) << 4));
             if constexpr (!AQ8) {
               const uint8_t* pa = pw + C::PKW;
 #pragma unroll
@@ -492,7 +532,8 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
                 const int v = it >> 3, u = it & 7;
                 const int r = (v & ~7) | ((v & 1) << 2) | ((v >> 1) & 3);
                 araw[jj * NITG + x] = *reinterpret_cast<const uint2*>(
-                    pa + r * 128 + (((4 * j + (u >> 1)) ^ (r & 7)) << 4) + ((u & 1) << 3));
+                    pa + (j >> 1) * (BT * 128) + r * 128 +
+                    (((4 * (j & 1) + (u >> 1)) ^ (r & 7)) << 4) + ((u & 1) << 3));
               }
             }
           }
@@ -549,8 +590,10 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
           tmem_st_wait();
           tc_fence_before();
         }
-        __syncwarp();
-        if (lane == 0) {
+        // every converter thread's writes are ordered before one elected arrival (fewer
+        // barrier events: each one wakes every suspended waiter of the CTA)
+        named_bar_sync(2, 128);
+        if (ct == 0) {
           mbar_arrive(smem_u32(&pk_empty[st]));
           if constexpr (C::GPB != 1) {
             mbar_arrive(smem_u32(&x_full[q % C::NXU]));
@@ -570,10 +613,16 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
   } else if (warp >= C::EPI0) {
     // ------------------------------------------------------------ epilogue
     const int et = threadIdx.x - 32 * C::EPI0;
-    const int h = (warp - C::EPI0) >> 2;           // column block (64 columns) of this warp
+    const int ew = (warp - C::EPI0) >> 2;
+    const int h = C::TEAMS == 1 ? ew : 0;          // column block (64 columns) of this warp
+    const int team = C::TEAMS == 2 ? ew : 0;       // hand-off units u with u % 2 == team
     const int row = 32 * (warp & 3) + lane;        // TMEM lane = weight row in the tile
     const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
     constexpr int NE = C::EPI_WARPS * 32;
+    // the tile flush: the whole epilogue, or the first team alone (barrier 5)
+    constexpr int NF = C::TEAMS == 2 ? 128 : NE;
+    constexpr uint32_t FB = C::TEAMS == 2 ? 5 : 1;
+    const uint32_t TB = 3 + team;                  // this team's unit barrier
     const int M = args.M, N = args.N;
     const bool sa_vec = args.sa_vec != 0, sw_vec = args.sw_vec != 0;
 
@@ -585,9 +634,10 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
       const int mt = (sg.t / args.tiles_n) * BT + et;
       const int nn = (sg.t % args.tiles_n) * C::BM + row;
       if (et < BT && mt < M)
-        sa = load_scale_block(args.sa, (size_t)mt * args.G, gb8, sg.gb, sg.ge, sa_vec, 128);
+        sa = load_scale_block(args.sa, (size_t)mt * args.G, gb8, sg.gb, sg.ge, sa_vec, 1, 0);
       if (nn < N)
-        sw = load_scale_block(args.sw, (size_t)nn * args.Gw, gb8, sg.gb, sg.ge, sw_vec, args.gw);
+        sw = load_scale_block(args.sw, (size_t)nn * args.Gw, gb8, sg.gb, sg.ge, sw_vec,
+                              args.gw / 128, args.gpg_shift);
     };
 
     float2 acc[C::CPT / 2];
@@ -636,10 +686,22 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
           const int r = (gb8 + j - sg.gb) % C::GPB;   // position in its hand-off unit
           const bool unit_last = r == C::GPB - 1 || gb8 + j == sg.ge - 1;
           const int sl = (u % C::NDU) * C::GPB + r;
+          if (C::TEAMS == 2 && (u & 1) != team) {   // the other team's unit
+            if (unit_last) ++u;
+            continue;
+          }
           if (r == 0) {
-            ok = mbar_wait(smem_u32(&g_done[u % C::NXU]), (uint32_t)(u / C::NXU) & 1u, lim,
-                           abort_flag);
-            ok = __all_sync(0xffffffffu, ok);
+            if constexpr (C::GPB == 1) {
+              ok = mbar_wait(smem_u32(&g_done[u % C::NXU]), (uint32_t)(u / C::NXU) & 1u, lim,
+                             abort_flag);
+              ok = __all_sync(0xffffffffu, ok);
+            } else {
+              // one warp of the team waits; the others park in the team's hardware barrier
+              if ((et & 127) < 32)
+                ok = mbar_wait(smem_u32(&g_done[u % C::NXU]), (uint32_t)(u / C::NXU) & 1u,
+                               lim, abort_flag);
+              ok = !bar_red_or(TB, 128, !ok);   // one decision for the team
+            }
             if (!ok) break;
             if (et == 0) trace_stamp(args, 7, i);
             tc_fence_after();
@@ -701,8 +763,13 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
           }
           if (unit_last) {
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&d_empty[u % C::NDU]));
+            if constexpr (C::GPB == 1) {
+              __syncwarp();
+              if (lane == 0) mbar_arrive(smem_u32(&d_empty[u % C::NDU]));
+            } else {
+              named_bar_sync(TB, 128);   // the team is done with the unit: one arrival
+              if ((et & 127) == 0) mbar_arrive(smem_u32(&d_empty[u % C::NDU]));
+            }
             ++u;
           }
           if (et == 0) trace_stamp(args, 3, i);
@@ -715,7 +782,23 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
       if (et == 0) trace_stamp(args, 15, 4 * k);
       aborted = aborted || bar_red_or(1, NE, !ok);
       if (aborted) break;
-      if constexpr (!DUMP) {
+      if constexpr (C::TEAMS == 2 && !DUMP) {
+        // the second team hands its sums to the first, which adds them (fixed order)
+        if (team == 1) {
+#pragma unroll
+          for (int e = 0; e < C::CPT; ++e)
+            s_red[e * C::BM + row] = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
+        }
+        bar_red_or(1, NE, false);
+        if (team == 0) {
+#pragma unroll
+          for (int e = 0; e < C::CPT; e += 2) {
+            acc[e / 2].x += s_red[e * C::BM + row];
+            acc[e / 2].y += s_red[(e + 1) * C::BM + row];
+          }
+        }
+      }
+      if (!DUMP && team == 0) {
         if (hoist) {
           const float2 sh = make_float2(sw_hoisted, sw_hoisted);
 #pragma unroll
@@ -731,45 +814,43 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
             if (m < M && nvalid) args.y[(size_t)m * N + n] = __float2half_rn(v);
           }
         } else {
-          // partial slot: 0 for this CTA's first tile, 1 for its last (a CTA shares at most
-          // those two tiles with other CTAs)
-          auto slot_of = [&](int c) -> size_t {
-            const int tf = sk_u0(args, c) / args.S;
-            return ((size_t)c * 2 + (sg.t == tf ? 0 : 1)) * (size_t)(BT * C::BM);
-          };
-          float* mine = args.part + slot_of(blockIdx.x);
+          // A split tile is finished by its owner, the CTA holding the tile's first stage:
+          // that is always the owner's last segment, so the others (the CTAs after it, for
+          // which the tile is their first segment) have published their parts by then or
+          // are about to.  A non-owner stores its fp32 part in its one slot and counts
+          // itself in; the owner waits for the count, then adds the parts in CTA order.
+          if ((int)blockIdx.x != cf) {
+            float* mine = args.part + (size_t)blockIdx.x * (BT * C::BM);
 #pragma unroll
-          for (int e = 0; e < C::CPT; ++e) {
-            const int ml = h * 64 + e;
-            mine[(size_t)ml * C::BM + row] = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
-          }
-          // publish: the barrier collects every thread's stores, one thread releases them
-          // with the arrival; the last arrival acquires everyone's before the sum
-          bar_red_or(1, NE, false);
-          if (et == 0) trace_stamp(args, 15, 4 * k + 1);
-          if (et == 0) {
-            fence_acq_rel_gpu();
-            const unsigned old = atomicAdd(&args.counters[sg.t], 1u);
-            const int last = old == (unsigned)(cl - cf);
-            if (last) fence_acq_rel_gpu();
-            *reinterpret_cast<volatile int*>(s_last) = last;
-          }
-          bar_red_or(1, NE, false);
-          if (et == 0) trace_stamp(args, 15, 4 * k + 2);
-          if (*reinterpret_cast<volatile int*>(s_last)) {
-            // the contributions, added in CTA order whoever arrives last; NCH CTAs' values
-            // are in flight at once
-            constexpr int NCH = 2;
+            for (int e = 0; e < C::CPT; ++e) {
+              const int ml = h * 64 + e;
+              mine[(size_t)ml * C::BM + row] = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
+            }
+            // the barrier collects every thread's stores; one thread releases them with
+            // the count
+            bar_red_or(FB, NF, false);
+            if (et == 0) trace_stamp(args, 15, 4 * k + 1);
+            if (et == 0) {
+              fence_acq_rel_gpu();
+              atomicAdd(&args.counters[sg.t], 1u);
+            }
+          } else {
+            if (et == 0) {
+              const unsigned need = (unsigned)(cl - cf);
+              ok = counter_wait(&args.counters[sg.t], need, lim, abort_flag);
+              trace_stamp(args, 15, 4 * k + 2);
+            }
+            aborted = bar_red_or(FB, NF, !ok);   // the other parts are visible to every thread
+            if (aborted) break;
+            // the other parts, added to this CTA's own in CTA order, NCH CTAs in flight
+            constexpr int NCH = C::CPT >= 64 ? 1 : C::CPT >= 32 ? 2 : 4;
+            for (int c = cf + 1; c <= cl; c += NCH) {
 #pragma unroll
-            for (int e0 = 0; e0 < C::CPT; e0 += 16) {
-              float sum[16];
-#pragma unroll
-              for (int e = 0; e < 16; ++e) sum[e] = 0.0f;
-              for (int c = cf; c <= cl; c += NCH) {
+              for (int e0 = 0; e0 < C::CPT; e0 += 16) {
                 float v[NCH][16];
 #pragma unroll
                 for (int cc = 0; cc < NCH; ++cc) {
-                  const float* src = args.part + slot_of(min(c + cc, cl));
+                  const float* src = args.part + (size_t)min(c + cc, cl) * (BT * C::BM);
 #pragma unroll
                   for (int e = 0; e < 16; ++e)
                     v[cc][e] = c + cc <= cl
@@ -779,15 +860,19 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
 #pragma unroll
                 for (int cc = 0; cc < NCH; ++cc)
 #pragma unroll
-                  for (int e = 0; e < 16; ++e) sum[e] += v[cc][e];
-              }
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const int m = m0 + h * 64 + e0 + e;
-                if (m < M && nvalid) args.y[(size_t)m * N + n] = __float2half_rn(sum[e]);
+                  for (int e = 0; e < 16; e += 2) {
+                    acc[(e0 + e) / 2].x += v[cc][e];
+                    acc[(e0 + e) / 2].y += v[cc][e + 1];
+                  }
               }
             }
-            if (et == 0) atomicExch(&args.counters[sg.t], 0u);
+#pragma unroll
+            for (int e = 0; e < C::CPT; ++e) {
+              const int m = m0 + h * 64 + e;
+              const float val = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
+              if (m < M && nvalid) args.y[(size_t)m * N + n] = __float2half_rn(val);
+            }
+            if (et == 0) args.counters[sg.t] = 0u;   // nobody else touches it in this launch
           }
         }
       }

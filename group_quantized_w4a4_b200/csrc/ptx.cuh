@@ -84,17 +84,22 @@ __device__ __forceinline__ uint64_t clock_cycles() {
 // i.e. at most the limit at clocks up to 2 GHz), or when *abort_flag becomes non-zero.
 // Each unsuccessful attempt sleeps in hardware for at most 1 ms (or until the phase
 // completes), so the limit and the abort word are checked at least every millisecond.
+// A suspended try_wait also resumes whenever any other barrier of the CTA changes, so the
+// loop runs once per such event; the abort word and the clock are only checked every 16th
+// time round, to keep those spurious rounds cheap.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
                                           volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = clock_cycles();
   for (uint32_t spin = 1;; ++spin) {
     if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
-    if (*abort_flag) return false;
-    if (clock_cycles() - t0 > 2 * limit_ns || spin > (1u << 30)) {
-      atomicOr(&g_device_status, DEV_TIMEOUT);
-      *abort_flag = 1;
-      return false;
+    if ((spin & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (clock_cycles() - t0 > 2 * limit_ns || spin > (1u << 30)) {
+        atomicOr(&g_device_status, DEV_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
     }
   }
 }
@@ -115,6 +120,27 @@ __device__ __forceinline__ bool mbar_wait2(uint32_t a, uint32_t pa, uint32_t b, 
 // earlier writes (cumulativity), so one thread can publish a CTA's results.
 __device__ __forceinline__ void fence_acq_rel_gpu() {
   asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+// Waits until the 32-bit counter at `p` (in global memory, written by other CTAs of this
+// grid with release semantics) equals `target`, with acquire semantics.  Bounded like
+// mbar_wait: gives up after about `limit_ns` or when *abort_flag is set, recording a
+// timeout in the device status word.
+__device__ __forceinline__ bool counter_wait(const unsigned* p, unsigned target,
+                                             uint64_t limit_ns, volatile int* abort_flag) {
+  const uint64_t t0 = clock_cycles();
+  for (uint32_t spin = 0;; ++spin) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    if (v == target) return true;
+    if (*abort_flag) return false;
+    if (clock_cycles() - t0 > 2 * limit_ns || spin > (1u << 30)) {
+      atomicOr(&g_device_status, DEV_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+    __nanosleep(64);
+  }
 }
 
 // Programmatic dependent launch.  grid_dep_wait() returns once the grid this one depends on
@@ -253,6 +279,11 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
 
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Named barrier over `nthreads` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Named barrier over `nthreads` threads that also ORs a predicate across them.

@@ -157,7 +157,7 @@ const char *apex_status_string(apex_status_t status);
 
 /*
  * Test hook: the next GEMM launch on this host thread skips the bulk copy of pipeline stage
- * `step` (a pair of K-groups, counted within each CTA), so its consumers wait until the
+ * `step` (two or four K-groups, counted within each CTA), so its consumers wait until the
  * time limit.  -1 turns it off.  Used only to test the timeout path; never needed by callers.
  */
 void apex_debug_withhold_step(int32_t step);
