@@ -154,11 +154,16 @@ class ClockSampler:
 EXPANDED_MIN_M = 128   # from this many tokens on, the step uses the expanded activation form
 
 
+def activation_form(M: int) -> str:
+    return "expanded" if M >= EXPANDED_MIN_M else "packed"
+
+
 class Problem:
     """Device-resident operands for one workload, in C copies (inputs larger than L2)."""
 
     def __init__(self, apex, torch, g: synth.Gemm, copies: int):
-        self.expanded = g.M >= EXPANDED_MIN_M
+        self.form = activation_form(g.M)
+        self.expanded = self.form == "expanded"
         self.g = g
         a, w = synth.make(g)
         self.a_host = a
@@ -311,7 +316,7 @@ def recorded_traffic(name: str):
 def roofline_obj(g, gemm_ms_avg, peaks, peaks_kind, traffic=None):
     hbm = float(peaks["hbm_gbs"]) * 1e9
     i8 = float(peaks.get("bf16_tflops", 1590.0)) * 1e12 * INT8_PER_BF16
-    nbytes = g.gemm_bytes(g.M >= EXPANDED_MIN_M)
+    nbytes = g.gemm_bytes(activation_form(g.M))
     t_bound, bound = roofline.bound_time_s(g.ops, nbytes, i8, hbm)
     t = gemm_ms_avg * 1e-3
     if bound == "hbm":
@@ -388,13 +393,13 @@ def run_apex(args, rank, world, local):
         extra[SECOND_WORKLOAD] = {
             "value": round(world * g2.ops / (ms2 * 1e-3) / 1e12, 2), "unit": "TOPS",
             "ms_per_step": round(ms2, 4),
-            "activation_form": "expanded" if g2.M >= EXPANDED_MIN_M else "packed",
+            "activation_form": activation_form(g2.M),
             "quantize_ms": round(qm2, 5), "gemm_ms": round(gm2, 5),
             "roofline": roofline_obj(g2, gm2, peaks, peaks_kind)}
         del p2
     if rank != 0:
         return None
-    expd = g.M >= EXPANDED_MIN_M
+    form = activation_form(g.M)
     line = {
         "metric": "W4A4-g128 GEMM effective TOPS (quantize + GEMM step) and % of roofline",
         "value": round(value, 2), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
@@ -403,7 +408,7 @@ def run_apex(args, rank, world, local):
         "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights, fp16)",
         "config": {"workload": g.name, "M": g.M, "N": g.N, "K": g.K, "group_a": 128,
                    "group_w": g.gw, "parallelism": f"replicas x{world}",
-                   "activation_form": "expanded" if g.M >= EXPANDED_MIN_M else "packed",
+                   "activation_form": form,
                    "l2": f"inputs larger than L2: {p_copies(g, l2)} rotating copies"},
         "roofline": roofline_obj(g, gemm_avg, peaks, peaks_kind),
         "e2e": {"value": round(world * g.ops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
@@ -413,9 +418,9 @@ def run_apex(args, rank, world, local):
         "launch": ("one CUDA graph of the K timed steps (eager warm-up), kernels launched as "
                    "programmatic dependents; per-kernel times from two more graphs of K "
                    "launches of that kernel alone"),
-        "gemm": {"kernel_ms": round(gemm_avg, 5), "bytes": g.gemm_bytes(expd)},
-        "quantize": {"kernel_ms": round(quant_avg, 5), "bytes": g.quant_bytes(expd),
-                     "GB/s": round(g.quant_bytes(expd) / (quant_avg * 1e-3) / 1e9, 1)},
+        "gemm": {"kernel_ms": round(gemm_avg, 5), "bytes": g.gemm_bytes(form)},
+        "quantize": {"kernel_ms": round(quant_avg, 5), "bytes": g.quant_bytes(form),
+                     "GB/s": round(g.quant_bytes(form) / (quant_avg * 1e-3) / 1e9, 1)},
         "clocks": clk,
         "impl": "apex",
     }
@@ -448,11 +453,11 @@ def run_sweep(args, rank, world, local):
         gm, qm = max_over_ranks(gm, world), max_over_ranks(qm, world)
         lines.append({
             "sweep": name, "M": g.M, "N": g.N, "K": g.K, "group_a": 128, "group_w": g.gw,
-            "steps": steps, "activation_form": "expanded" if g.M >= EXPANDED_MIN_M else "packed",
+            "steps": steps, "activation_form": activation_form(g.M),
             "step_ms": round(ms, 5), "gemm_ms": round(gm, 5), "quantize_ms": round(qm, 5),
             "step_TOPS": round(world * g.ops / (ms * 1e-3) / 1e12, 2),
             "gemm_TOPS": round(g.ops / (gm * 1e-3) / 1e12, 2),
-            "gemm_GBs": round(g.gemm_bytes(g.M >= EXPANDED_MIN_M) / (gm * 1e-3) / 1e9, 1),
+            "gemm_GBs": round(g.gemm_bytes(activation_form(g.M)) / (gm * 1e-3) / 1e9, 1),
             "roofline": roofline_obj(g, gm, peaks, peaks_kind)})
     return lines if rank == 0 else None
 

@@ -81,6 +81,10 @@ def load_library(build_if_missing: bool = True):
         lib.apex_w4a4_gemm_noalloc.restype = st
         lib.apex_w4a4_gemm_workspace_size.argtypes = [I64, I64, I64, I32, I32]
         lib.apex_w4a4_gemm_workspace_size.restype = SZ
+        lib.apex_w4a4_linear.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, SZ, P]
+        lib.apex_w4a4_linear.restype = st
+        lib.apex_w4a4_linear_workspace_size.argtypes = [I64, I64, I64, I32, I32]
+        lib.apex_w4a4_linear_workspace_size.restype = SZ
         lib.apex_w4a4_group_partials.argtypes = [I64, I64, I64, P, P, P, P]
         lib.apex_w4a4_group_partials.restype = st
         lib.apex_get_device_status.argtypes = [P]
@@ -195,6 +199,21 @@ def apex_w4a4_gemm_workspace_size(M, N, K, group_a, group_w) -> int:
     return int(load_library().apex_w4a4_gemm_workspace_size(M, N, K, group_a, group_w))
 
 
+def apex_w4a4_linear(M, N, K, group_a, group_w, x_f16, w_packed, w_scales, y_f16,
+                     workspace=None, workspace_bytes=None, stream=None):
+    if workspace is not None and workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(load_library().apex_w4a4_linear(M, N, K, group_a, group_w, _ptr(x_f16),
+                                           _ptr(w_packed), _ptr(w_scales), _ptr(y_f16),
+                                           _ptr(workspace), workspace_bytes or 0,
+                                           _stream(stream)),
+           "apex_w4a4_linear")
+
+
+def apex_w4a4_linear_workspace_size(M, N, K, group_a, group_w) -> int:
+    return int(load_library().apex_w4a4_linear_workspace_size(M, N, K, group_a, group_w))
+
+
 def apex_w4a4_group_partials(M, N, K, a_packed, w_packed, partials_i32, stream=None):
     _check(load_library().apex_w4a4_group_partials(M, N, K, _ptr(a_packed), _ptr(w_packed),
                                                    _ptr(partials_i32), _stream(stream)),
@@ -242,10 +261,12 @@ def pack_weights(w, group_w: int = 128, stream=None):
     return packed, scales
 
 
-def workspace(M, N, K, group_a=128, group_w=128, device="cuda"):
-    """A zero-filled workspace of the size apex_w4a4_gemm uses for this problem (or None)."""
+def workspace(M, N, K, group_a=128, group_w=128, device="cuda", linear=False):
+    """A zero-filled workspace of the size apex_w4a4_gemm (or, with linear=True,
+    apex_w4a4_linear) uses for this problem (or None)."""
     import torch
-    nbytes = apex_w4a4_gemm_workspace_size(M, N, K, group_a, group_w)
+    size_fn = apex_w4a4_linear_workspace_size if linear else apex_w4a4_gemm_workspace_size
+    nbytes = size_fn(M, N, K, group_a, group_w)
     if nbytes == 0:
         return None
     return torch.zeros(nbytes, dtype=torch.uint8, device=device)

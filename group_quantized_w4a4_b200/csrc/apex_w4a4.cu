@@ -298,6 +298,17 @@ apex_status_t quantize_launch(const void* x, int64_t rows, int64_t K, int32_t gr
   return cuda_status(cudaPeekAtLastError());
 }
 
+// apex_w4a4_linear: the activation form the quantizer writes for a batch of M tokens
+// (expanded from 128 tokens on, where activation bytes are small next to the math).
+constexpr int64_t kLinearExpandedMinM = 128;
+
+size_t linear_act_bytes(int64_t M, int64_t K) {   // quantized activations + their scales
+  const int64_t per_row = M >= kLinearExpandedMinM ? K : K / 2;
+  const size_t a = (((size_t)M * (size_t)per_row) + 255) & ~(size_t)255;
+  const size_t sc = (((size_t)M * (size_t)(K / 128) * 2) + 255) & ~(size_t)255;
+  return a + sc;
+}
+
 }  // namespace
 
 extern "C" {
@@ -342,6 +353,37 @@ apex_status_t apex_w4a4_gemm_expanded(int64_t M, int64_t N, int64_t K, int32_t g
       !make_expanded_map(&maps.a, a_q8, M, K, p.bt))
     return APEX_ERR_CUDA;
   return launch_gemm<apex::MODE_AQ8>(p, maps, a, static_cast<cudaStream_t>(stream));
+}
+
+size_t apex_w4a4_linear_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                       int32_t group_w) {
+  if (check_gemm_args(M, N, K, group_a, group_w) != APEX_OK) return 0;
+  return linear_act_bytes(M, K) + workspace_for(make_plan(M, N, K, true));
+}
+
+apex_status_t apex_w4a4_linear(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                               int32_t group_w, const void* x_f16, const void* w_packed,
+                               const void* w_scales, void* y_f16, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  apex_status_t st = check_gemm_args(M, N, K, group_a, group_w);
+  if (st != APEX_OK) return st;
+  if (!x_f16 || !w_packed || !w_scales || !y_f16) return APEX_ERR_INVALID_ARG;
+  if (!aligned(x_f16, 16) || !aligned(w_packed, 16) || !aligned(w_scales, 2) ||
+      !aligned(y_f16, 2) || (workspace && !aligned(workspace, 256)))
+    return APEX_ERR_ALIGNMENT;
+  const size_t act = linear_act_bytes(M, K);
+  if (!workspace || workspace_bytes < act) return APEX_ERR_INVALID_ARG;
+  const bool expanded = M >= kLinearExpandedMinM;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* a_q = ws;
+  void* a_sc = ws + ((((size_t)M * (size_t)(expanded ? K : K / 2)) + 255) & ~(size_t)255);
+  st = quantize_launch(x_f16, M, K, 128, a_q, a_sc, stream, expanded);
+  if (st != APEX_OK) return st;
+  return expanded ? apex_w4a4_gemm_expanded(M, N, K, group_a, group_w, a_q, a_sc, w_packed,
+                                            w_scales, y_f16, ws + act, workspace_bytes - act,
+                                            stream)
+                  : apex_w4a4_gemm(M, N, K, group_a, group_w, a_q, a_sc, w_packed, w_scales,
+                                   y_f16, ws + act, workspace_bytes - act, stream);
 }
 
 size_t apex_w4a4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group_a,

@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
   // is free again and its partial is in tensor memory (one commit serves both waiters)
   uint64_t* g_done = x_full + C::NXU;
   uint64_t* d_empty = g_done + C::NXU;
-  uint64_t* mma_done = d_empty + C::NSLOT;
+  uint64_t* mma_done = d_empty + C::NDU;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* s_abort = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
   int* s_last = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);

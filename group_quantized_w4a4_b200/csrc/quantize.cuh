@@ -29,6 +29,11 @@ __device__ __forceinline__ float absmax8(const uint4& v) {
   return fmaxf(__low2float(m), __high2float(m));
 }
 
+// The group's stored scale: fp16_rne(fp32(absmax) / 7), IEEE fp32 division.
+__device__ __forceinline__ __half group_scale(float absmax) {
+  return __float2half_rn(__fdiv_rn(absmax, 7.0f));
+}
+
 // Quantize 8 fp16 values against scale sf (fp32 copy of the stored fp16 scale) and pack
 // them into 4 bytes (little-endian: element 0 in the low nibble of byte 0).
 __device__ __forceinline__ uint32_t quant_pack8(const uint4& v, float sf) {
@@ -99,7 +104,7 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __rest
 #pragma unroll
       for (int off = 8; off >= 1; off >>= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-      const __half s = __float2half_rn(__fdiv_rn(amax, 7.0f));
+      const __half s = group_scale(amax);
       const float sf = __half2float(s);
       if (live) {
 #pragma unroll
@@ -119,7 +124,7 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __rest
 #pragma unroll
       for (int off = 8; off >= 1; off >>= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-      const __half s = __float2half_rn(__fdiv_rn(amax, 7.0f));
+      const __half s = group_scale(amax);
       const float sf = __half2float(s);
       if (live) {
         for (int c = 0; c < chunks; ++c) {

@@ -79,18 +79,19 @@ class Gemm:
     def ops(self) -> float:
         return 2.0 * self.M * self.N * self.K
 
-    def gemm_bytes(self, expanded: bool = False) -> int:
-        """Algorithmic HBM bytes of one GEMM call: A (packed, or one byte per element in the
-        expanded form) and packed W, fp16 scales, fp16 Y."""
+    def gemm_bytes(self, form: str = "packed") -> int:
+        """Algorithmic HBM bytes of one GEMM call: A, packed W, fp16 scales, fp16 Y.  A is
+        packed int4 plus scales ("packed") or one byte per element plus scales
+        ("expanded")."""
         M, N, K = self.M, self.N, self.K
-        a = M * K if expanded else M * K // 2
-        return (a + N * K // 2 + 2 * M * (K // self.ga)
-                + 2 * N * (K // self.gw) + 2 * M * N)
+        a = {"packed": M * K // 2 + 2 * M * (K // self.ga),
+             "expanded": M * K + 2 * M * (K // self.ga)}[form]
+        return a + N * K // 2 + 2 * N * (K // self.gw) + 2 * M * N
 
-    def quant_bytes(self, expanded: bool = False) -> int:
+    def quant_bytes(self, form: str = "packed") -> int:
         """Algorithmic HBM bytes of the online activation quantizer."""
         M, K = self.M, self.K
-        return 2 * M * K + (M * K if expanded else M * K // 2) + 2 * M * (K // self.ga)
+        return 2 * M * K + (M * K if form == "expanded" else M * K // 2) + 2 * M * (K // self.ga)
 
 
 def workloads() -> dict:

@@ -127,6 +127,26 @@ apex_status_t apex_w4a4_gemm_noalloc(int64_t M, int64_t N, int64_t K, int32_t gr
                                      const void *w_packed, const void *w_scales, void *y_f16,
                                      void *stream);
 
+/*
+ * Online quantization and the W4A4 GEMM in one call: y_f16[M][N] from fp16 activations
+ * x_f16 [M][K] (row-major, 16-byte aligned) and packed weights.  The activations are
+ * quantized with exactly the rule of apex_quantize_act_int4 (group_a = 128) into the
+ * workspace (packed below 128 tokens, the expanded form from 128 tokens on), then the GEMM
+ * runs on them: the result equals apex_quantize_act_int4 followed by apex_w4a4_gemm.
+ * workspace: at least apex_w4a4_linear_workspace_size(...) bytes (else
+ *   APEX_ERR_INVALID_ARG), 256-byte aligned; its tail is the GEMM's split-K scratch, with
+ *   apex_w4a4_gemm's zero-counter contract (zero it once before the first call).
+ * The same group rules, alignment rules and errors as apex_w4a4_gemm otherwise.
+ */
+apex_status_t apex_w4a4_linear(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                               int32_t group_w, const void *x_f16, const void *w_packed,
+                               const void *w_scales, void *y_f16, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
+/* Workspace bytes apex_w4a4_linear needs for this problem (0 when it needs none). */
+size_t apex_w4a4_linear_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                       int32_t group_w);
+
 /* Workspace bytes apex_w4a4_gemm would use for this problem (0 when it needs none). */
 size_t apex_w4a4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group_a,
                                      int32_t group_w);

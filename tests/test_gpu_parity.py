@@ -335,6 +335,74 @@ def test_gemm_expanded_large_sampled_rows(apex, name):
     assert_close(host(y)[rows].astype(np.float64), ref)
 
 
+# ------------------------------------------------------------------ quantize + GEMM in one call
+
+
+def run_linear(apex, x, wp, sw, M, N, K, gw):
+    y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+    w = apex.workspace(M, N, K, 128, gw, linear=True)
+    apex.apex_w4a4_linear(M, N, K, 128, gw, dev(x), dev(wp), dev(sw), y, w)
+    torch.cuda.synchronize()
+    check_status(apex)
+    return y
+
+
+@pytest.mark.parametrize("M,N,K,gw", [(1, 256, 512, 128), (5, 384, 1024, 128),
+                                      (16, 256, 512, 128), (16, 1024, 2048, 512),
+                                      (17, 300, 1024, 128), (32, 512, 4096, 128),
+                                      (48, 256, 1024, 1024), (64, 640, 2048, 128),
+                                      (65, 256, 768, 128), (200, 384, 1024, 256)])
+def test_linear_matches_oracle_and_two_step_path(apex, M, N, K, gw):
+    """apex_w4a4_linear (quantize into its workspace, then the GEMM): within tolerance of the
+    oracle and bit-identical to the separate quantize and GEMM calls."""
+    a = synth.activations(M, K, "outlier", 5 * M + K)
+    w = synth.weights(N, K, 5 * N + K)
+    ap, sa = oracle.quantize_pack(a, 128)
+    wp, sw = oracle.quantize_pack(w, gw)
+    ref = oracle.gemm(ap, sa, wp, sw, M, N, K, 128, gw)
+    y = run_linear(apex, a, wp, sw, M, N, K, gw)
+    assert_close(host(y).astype(np.float64), ref)
+    if M >= 128:
+        q8, sa2 = apex.quantize_act_expanded(dev(a), 128)
+        y2 = torch.empty((M, N), dtype=torch.float16, device="cuda")
+        apex.apex_w4a4_gemm_expanded(M, N, K, 128, gw, q8, sa2, dev(wp), dev(sw), y2,
+                                     apex.workspace(M, N, K, 128, gw))
+    else:
+        ap2, sa2 = apex.quantize_act(dev(a), 128)
+        y2 = torch.empty((M, N), dtype=torch.float16, device="cuda")
+        apex.apex_w4a4_gemm(M, N, K, 128, gw, ap2, sa2, dev(wp), dev(sw), y2,
+                            apex.workspace(M, N, K, 128, gw))
+    torch.cuda.synchronize()
+    check_status(apex)
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+
+
+def test_linear_decode_workload_and_edge_values(apex):
+    """The decode workload end to end, and a batch with all-zero, tiny and tie-valued rows."""
+    g = synth.workloads()["decode_m16_n8192_k8192"]
+    a, w = synth.make(g)
+    a[3] = 0.0                                   # all-zero rows: scale 0, q = 0
+    a[4, :] = np.float16(1e-7)                   # scale underflows to fp16 zero
+    a[5, :128] = np.float16(7.0)                 # s = 1 exactly, then ties
+    a[5, 0:8] = np.array([0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.5, -3.5], dtype=np.float16)
+    wp, sw = oracle.quantize_pack(w, g.gw)
+    ap, sa = oracle.quantize_pack(a, 128)
+    ref = oracle.gemm(ap, sa, wp, sw, g.M, g.N, g.K, 128, g.gw)
+    y = run_linear(apex, a, wp, sw, g.M, g.N, g.K, g.gw)
+    assert_close(host(y).astype(np.float64), ref)
+
+
+def test_linear_refuses_a_missing_workspace(apex):
+    M, N, K = 16, 256, 512
+    x = torch.zeros((M, K), dtype=torch.float16, device="cuda")
+    wp = torch.zeros((N, K // 2), dtype=torch.uint8, device="cuda")
+    sw = torch.zeros((N, K // 128), dtype=torch.float16, device="cuda")
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    with pytest.raises(apex.ApexError) as e:
+        apex.apex_w4a4_linear(M, N, K, 128, 128, x, wp, sw, y, None)
+    assert e.value.code == apex.APEX_ERR_INVALID_ARG
+
+
 # ------------------------------------------------------------------ failure path
 
 
