@@ -70,6 +70,12 @@ def barrier(world):
         dist.barrier()
 
 
+def job_throughput(ops_per_step: float, ms_per_step: float, world: int) -> float:
+    """Whole-job TOPS: every replica ran ops_per_step per step; the step time is the
+    slowest rank's."""
+    return world * ops_per_step / (ms_per_step * 1e-3) / 1e12
+
+
 def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
@@ -378,7 +384,7 @@ def run_apex(args, rank, world, local):
                                                           args.warmup, world, l2, clocks)
     ms_step = max_over_ranks(total_ms / args.steps, world)
     gemm_avg = max_over_ranks(gemm_avg, world)
-    value = world * g.ops / (ms_step * 1e-3) / 1e12
+    value = job_throughput(g.ops, ms_step, world)
     e2e_ms, hb, db = e2e_workload(apex, torch, g, max(3, args.steps), args.warmup, p)
     e2e_ms = max_over_ranks(e2e_ms, world)
     del p
@@ -391,7 +397,7 @@ def run_apex(args, rank, world, local):
         gm2, qm2 = max_over_ranks(gm2, world), max_over_ranks(qm2, world)
         ms2 = max_over_ranks(tot2 / max(3, args.steps // 4), world)
         extra[SECOND_WORKLOAD] = {
-            "value": round(world * g2.ops / (ms2 * 1e-3) / 1e12, 2), "unit": "TOPS",
+            "value": round(job_throughput(g2.ops, ms2, world), 2), "unit": "TOPS",
             "ms_per_step": round(ms2, 4),
             "activation_form": activation_form(g2.M),
             "quantize_ms": round(qm2, 5), "gemm_ms": round(gm2, 5),
@@ -411,7 +417,7 @@ def run_apex(args, rank, world, local):
                    "activation_form": form,
                    "l2": f"inputs larger than L2: {p_copies(g, l2)} rotating copies"},
         "roofline": roofline_obj(g, gemm_avg, peaks, peaks_kind),
-        "e2e": {"value": round(world * g.ops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
+        "e2e": {"value": round(job_throughput(g.ops, e2e_ms, world), 3), "unit": "TOPS",
                 "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db,
                 "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": 2 * args.steps,
@@ -455,7 +461,7 @@ def run_sweep(args, rank, world, local):
             "sweep": name, "M": g.M, "N": g.N, "K": g.K, "group_a": 128, "group_w": g.gw,
             "steps": steps, "activation_form": activation_form(g.M),
             "step_ms": round(ms, 5), "gemm_ms": round(gm, 5), "quantize_ms": round(qm, 5),
-            "step_TOPS": round(world * g.ops / (ms * 1e-3) / 1e12, 2),
+            "step_TOPS": round(job_throughput(g.ops, ms, world), 2),
             "gemm_TOPS": round(g.ops / (gm * 1e-3) / 1e12, 2),
             "gemm_GBs": round(g.gemm_bytes(activation_form(g.M)) / (gm * 1e-3) / 1e9, 1),
             "roofline": roofline_obj(g, gm, peaks, peaks_kind)})

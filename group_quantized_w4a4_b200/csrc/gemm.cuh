@@ -108,22 +108,15 @@ __device__ __forceinline__ void trace_stamp(const GemmArgs& a, int role, int ste
 // boxes of packed weights), so the per-stage hand-off costs are spread over more MMAs.
 __host__ __device__ constexpr int stage_groups(int bt) { return bt <= 32 ? 4 : 2; }
 
-#ifndef APEX_WSM_MAX_BT
-#define APEX_WSM_MAX_BT 0
-#endif
-
 template <int BT, int MODE>
 struct GemmCfg {
   static constexpr bool AQ8 = MODE == MODE_AQ8;
-  // Narrow tiles keep the expanded weight tile in shared memory (both MMA operands from
-  // shared memory); wide tiles keep it in tensor memory.
-  static constexpr bool WSM = !AQ8 && BT <= APEX_WSM_MAX_BT;
   static constexpr int BM = 128;
   static constexpr int KPS = stage_groups(BT);                     // K-groups per packed stage
   static constexpr int NBOX = KPS / 2;                             // 128-byte boxes per stage
   // operand slots (per group): expanded weight tile (tensor or shared memory) + token tile
-  static constexpr int NX = WSM ? (BT <= 32 ? 6 : 4) : BT >= 128 ? (AQ8 ? 6 : 4) : 8;
-  static constexpr int NSLOT = WSM ? NX : BT >= 128 ? (AQ8 ? 2 : 3) : KPS == 4 ? 8 : 4;
+  static constexpr int NX = BT >= 128 ? (AQ8 ? 6 : 4) : 8;
+  static constexpr int NSLOT = BT >= 128 ? (AQ8 ? 2 : 3) : KPS == 4 ? 8 : 4;
   // Epilogue: 8 warps.  Wide tiles split the 128 columns in two halves; narrow tiles run
   // two teams of 4 warps that take alternate hand-off units (so one team's TMEM loads and
   // waits overlap the other's arithmetic) and add their sums at the end of a segment.
@@ -135,7 +128,7 @@ struct GemmCfg {
   static constexpr int EPI0 = CONV0 + 4 * CWG;     // first epilogue warp
   static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
   static constexpr int W_COL0 = 0;
-  static constexpr int D_COL0 = WSM ? 0 : NX * 32;
+  static constexpr int D_COL0 = NX * 32;
   static constexpr int TMEM_USED = D_COL0 + NSLOT * BT;
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
   static_assert(TMEM_USED <= 512, "tensor memory budget");
@@ -143,16 +136,14 @@ struct GemmCfg {
   static constexpr int PKA = AQ8 ? 0 : BT * 64 * KPS;   // [BT rows][128 B], 128-byte swizzle
   static constexpr int PK_STAGE = PKW + PKA;
   static constexpr int XA = BT * 128;                    // one group's int8 token tile
-  static constexpr int XW = WSM ? BM * 128 : 0;          // one group's int8 weight tile
   static constexpr int SAT = 2 * 8 * BT * 4;  // token scales: 2 blocks x [8 groups][BT] fp32
   static constexpr int RED = TEAMS == 2 ? CPT * BM * 4 : 0;   // second team's sums [CPT][BM]
-  static constexpr int FIXED = NX * (XA + XW) + SAT + RED + 4096;
+  static constexpr int FIXED = NX * XA + SAT + RED + 4096;
   static constexpr int NP_FIT = (200 * 1024 - FIXED) / PK_STAGE;
   static constexpr int NP = NP_FIT > 12 ? 12 : (NP_FIT < 2 ? 2 : NP_FIT);  // packed stages
   static constexpr int OFF_PK = 0;
   static constexpr int OFF_XA = OFF_PK + NP * PK_STAGE;
-  static constexpr int OFF_XW = OFF_XA + NX * XA;
-  static constexpr int OFF_SAT = OFF_XW + NX * XW;
+  static constexpr int OFF_SAT = OFF_XA + NX * XA;
   static constexpr int OFF_RED = OFF_SAT + SAT;
   static constexpr int OFF_BAR = OFF_RED + RED;
   // Hand-off unit: the groups that pass between converters, MMA and epilogue under one
@@ -174,7 +165,7 @@ struct GemmCfg {
   }
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
-  static_assert(PK_STAGE % 1024 == 0 && XA % 1024 == 0 && XW % 1024 == 0, "stage alignment");
+  static_assert(PK_STAGE % 1024 == 0 && XA % 1024 == 0, "stage alignment");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
@@ -280,7 +271,6 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* pk = smem + C::OFF_PK;
   uint8_t* xa = smem + C::OFF_XA;
-  uint8_t* xw = smem + C::OFF_XW;
   float* s_sat = reinterpret_cast<float*>(smem + C::OFF_SAT);
   float* s_red = reinterpret_cast<float*>(smem + C::OFF_RED);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -335,8 +325,8 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   // Launched as a programmatic dependent: the prologue above overlaps the previous grid's
-  // tail; no global memory is read or written before that grid has completed.
-  grid_dep_wait();
+  // tail.  The roles that touch global memory (producer, epilogue) wait for that grid
+  // before their first access; the producer first asks L2 for its first weight tiles.
   grid_dep_launch();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(s_tmem);
   volatile int* abort_flag = s_abort;
@@ -358,6 +348,13 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
     bool ok = true;
     Seg sg;
     if (lane == 0) trace_stamp_at(args, 5, 4);
+    if (lane == 0 && get_seg(args, 0, sg)) {
+      // L2 prefetches change no data, so they may run while the previous grid finishes
+      const int n0 = (sg.t % args.tiles_n) * C::BM;
+      for (int g = sg.gb, b = 0; g < sg.ge && b < 32; g += 2, ++b)
+        tma_prefetch_l2_2d(&tmW, g * 64, n0);
+    }
+    grid_dep_wait();
     for (int k = 0; ok && get_seg(args, k, sg); ++k) {
       if (lane == 0 && k == 0) trace_stamp_at(args, 5, 5);
       const int n0 = (sg.t % args.tiles_n) * C::BM;
@@ -441,18 +438,10 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
               const int xs = xu * C::GPB + t;
               const uint32_t d = tbase + C::D_COL0 + (du * C::GPB + t) * BT;
               const uint64_t b0 = smem_desc_k_sw128(smem_u32(xa + xs * C::XA));
-              if constexpr (C::WSM) {
-                const uint64_t a0 = smem_desc_k_sw128(smem_u32(xw + xs * C::XW));
+              const uint32_t a0 = tbase + C::W_COL0 + xs * 32;
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                  umma_i8_ss(d, a0 + (uint64_t)(j * 2), b0 + (uint64_t)(j * 2), idesc,
-                             j > 0 ? 1u : 0u);
-              } else {
-                const uint32_t a0 = tbase + C::W_COL0 + xs * 32;
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                  umma_i8_ts(d, a0 + j * 8, b0 + (uint64_t)(j * 2), idesc, j > 0 ? 1u : 0u);
-              }
+              for (int j = 0; j < 4; ++j)
+                umma_i8_ts(d, a0 + j * 8, b0 + (uint64_t)(j * 2), idesc, j > 0 ? 1u : 0u);
             }
             trace_stamp(args, 9, i + j0);
             umma_commit(smem_u32(&g_done[xu]));
@@ -543,18 +532,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
           const int j = cwg + C::CWG * jj;
           if (j >= nk) continue;
           const int xs = C::slot(q, i + j, j);
-          if constexpr (C::WSM) {
-            // the row's 128 expanded bytes, 16-byte chunk c at c ^ (row & 7)
-            uint8_t* wdst = xw + xs * C::XW + row * 128;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-              const uint4 a = wraw[4 * jj + cc];
-              *reinterpret_cast<uint4*>(wdst + (((2 * cc) ^ (row & 7)) << 4)) =
-                  make_uint4(expand_lo(a.x), expand_hi(a.x), expand_lo(a.y), expand_hi(a.y));
-              *reinterpret_cast<uint4*>(wdst + (((2 * cc + 1) ^ (row & 7)) << 4)) =
-                  make_uint4(expand_lo(a.z), expand_hi(a.z), expand_lo(a.w), expand_hi(a.w));
-            }
-          } else {
+          {
             uint32_t e0[16], e1[16];
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
@@ -586,10 +564,8 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
           }
         }
         if constexpr (!AQ8) fence_proxy_async_smem();
-        if constexpr (!C::WSM) {
-          tmem_st_wait();
-          tc_fence_before();
-        }
+        tmem_st_wait();
+        tc_fence_before();
         // every converter thread's writes are ordered before one elected arrival (fewer
         // barrier events: each one wakes every suspended waiter of the CTA)
         named_bar_sync(2, 128);
@@ -612,6 +588,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
     }
   } else if (warp >= C::EPI0) {
     // ------------------------------------------------------------ epilogue
+    grid_dep_wait();   // scales, outputs and split-K scratch are global memory
     const int et = threadIdx.x - 32 * C::EPI0;
     const int ew = (warp - C::EPI0) >> 2;
     const int h = C::TEAMS == 1 ? ew : 0;          // column block (64 columns) of this warp
