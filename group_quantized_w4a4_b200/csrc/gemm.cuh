@@ -123,7 +123,9 @@ struct GemmCfg {
   static constexpr int EPI_WARPS = 8;
   static constexpr int TEAMS = BT >= 128 ? 1 : 2;
   static constexpr int CPT = BT >= 128 ? 64 : BT;  // columns per epilogue thread
-  static constexpr int CWG = 1;                    // converter warpgroups
+  // converter warpgroups (a second one, with 18 warps, leaves 96 registers a thread and
+  // spills in the epilogue: slower)
+  static constexpr int CWG = 1;
   static constexpr int CONV0 = 2;                  // first converter warp
   static constexpr int EPI0 = CONV0 + 4 * CWG;     // first epilogue warp
   static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
@@ -136,7 +138,8 @@ struct GemmCfg {
   static constexpr int PKA = AQ8 ? 0 : BT * 64 * KPS;   // [BT rows][128 B], 128-byte swizzle
   static constexpr int PK_STAGE = PKW + PKA;
   static constexpr int XA = BT * 128;                    // one group's int8 token tile
-  static constexpr int SAT = 2 * 8 * BT * 4;  // token scales: 2 blocks x [8 groups][BT] fp32
+  // token scales: per team, 2 blocks x [8 groups][BT] fp32
+  static constexpr int SAT = 2 * TEAMS * 8 * BT * 4;
   static constexpr int RED = TEAMS == 2 ? CPT * BM * 4 : 0;   // second team's sums [CPT][BM]
   static constexpr int FIXED = NX * XA + SAT + RED + 4096;
   static constexpr int NP_FIT = (200 * 1024 - FIXED) / PK_STAGE;
@@ -297,10 +300,10 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NP; ++i) {
       mbar_init(smem_u32(&pk_full[i]), 1);
-      mbar_init(smem_u32(&pk_empty[i]), 1);   // one elected converter arrival
+      mbar_init(smem_u32(&pk_empty[i]), C::CWG);   // one elected arrival per warpgroup
     }
     for (int i = 0; i < C::NXU; ++i) {
-      mbar_init(smem_u32(&x_full[i]), 1);     // one elected converter arrival
+      mbar_init(smem_u32(&x_full[i]), C::CWG);     // one elected arrival per warpgroup
       mbar_init(smem_u32(&g_done[i]), 1);
     }
     for (int i = 0; i < C::NDU; ++i) {
@@ -326,7 +329,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
   tc_fence_after();
   // Launched as a programmatic dependent: the prologue above overlaps the previous grid's
   // tail.  The roles that touch global memory (producer, epilogue) wait for that grid
-  // before their first access; the producer first asks L2 for its first weight tiles.
+  // before their first access.
   grid_dep_launch();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(s_tmem);
   volatile int* abort_flag = s_abort;
@@ -348,12 +351,6 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
     bool ok = true;
     Seg sg;
     if (lane == 0) trace_stamp_at(args, 5, 4);
-    if (lane == 0 && get_seg(args, 0, sg)) {
-      // L2 prefetches change no data, so they may run while the previous grid finishes
-      const int n0 = (sg.t % args.tiles_n) * C::BM;
-      for (int g = sg.gb, b = 0; g < sg.ge && b < 32; g += 2, ++b)
-        tma_prefetch_l2_2d(&tmW, g * 64, n0);
-    }
     grid_dep_wait();
     for (int k = 0; ok && get_seg(args, k, sg); ++k) {
       if (lane == 0 && k == 0) trace_stamp_at(args, 5, 5);
@@ -461,6 +458,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
     // Warpgroup w expands the K-groups j of every stage with j % CWG == w, so with two
     // warpgroups both work on each stage at once, one group each.
     const int cwg = (warp - C::CONV0) >> 2;
+    const uint32_t CB = cwg == 0 ? 2 : 6;              // this warpgroup's named barrier
     const int row = 32 * (warp & 3) + lane;            // this thread's W row (TMEM lane)
     const int ct = threadIdx.x - 32 * (C::CONV0 + 4 * cwg);  // 0..127, for the token rows
     const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
@@ -491,7 +489,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
         }
         // one decision for the whole warpgroup, so none of it can be left at the barrier
         // below when another part gives up
-        ok = !bar_red_or(2, 128, !ok);
+        ok = !bar_red_or(CB, 128, !ok);
         tc_fence_after();   // tensor-memory writes below come after the slots' last reads
         if (!ok) break;
         if (lane == 0 && (warp & 3) == 2) trace_stamp(args, 4, q);
@@ -568,7 +566,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
         tc_fence_before();
         // every converter thread's writes are ordered before one elected arrival (fewer
         // barrier events: each one wakes every suspended waiter of the CTA)
-        named_bar_sync(2, 128);
+        named_bar_sync(CB, 128);
         if (ct == 0) {
           mbar_arrive(smem_u32(&pk_empty[st]));
           if constexpr (C::GPB != 1) {
@@ -600,6 +598,8 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
     constexpr int NF = C::TEAMS == 2 ? 128 : NE;
     constexpr uint32_t FB = C::TEAMS == 2 ? 5 : 1;
     const uint32_t TB = 3 + team;                  // this team's unit barrier
+    // token of this thread for the token-scale staging (each team stages its own copy)
+    const int tt = C::TEAMS == 2 ? (et & 127) : et;
     const int M = args.M, N = args.N;
     const bool sa_vec = args.sa_vec != 0, sw_vec = args.sw_vec != 0;
 
@@ -608,9 +608,9 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
       sa = make_uint4(0, 0, 0, 0);
       sw = make_uint4(0, 0, 0, 0);
       if (DUMP) return;
-      const int mt = (sg.t / args.tiles_n) * BT + et;
+      const int mt = (sg.t / args.tiles_n) * BT + tt;
       const int nn = (sg.t % args.tiles_n) * C::BM + row;
-      if (et < BT && mt < M)
+      if (tt < BT && mt < M)
         sa = load_scale_block(args.sa, (size_t)mt * args.G, gb8, sg.gb, sg.ge, sa_vec, 1, 0);
       if (nn < N)
         sw = load_scale_block(args.sw, (size_t)nn * args.Gw, gb8, sg.gb, sg.ge, sw_vec,
@@ -649,12 +649,14 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
           block_scales(nx, nx.gb & ~7, sa_n, sw_n);
         else
           sa_n = sw_n = make_uint4(0, 0, 0, 0);
-        float* sat = s_sat + buf * 8 * BT;
-        if (et < BT) {
+        float* sat = s_sat + (buf * C::TEAMS + team) * 8 * BT;
+        if (tt < BT) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) sat[j * BT + et] = half_of(sa_c, j);
+          for (int j = 0; j < 8; ++j) sat[j * BT + tt] = half_of(sa_c, j);
         }
-        aborted = bar_red_or(1, NE, !ok);   // token scales visible; one abort decision
+        // token scales visible, one abort decision: per team, so that the two teams do not
+        // wait for each other at every block (the segment end below joins them)
+        aborted = C::TEAMS == 2 ? bar_red_or(TB, 128, !ok) : bar_red_or(1, NE, !ok);
         if (aborted) break;
         if (gb8 <= sg.gb) sw_hoisted = half_of(sw_c, sg.gb - gb8) * (1.0f / 256.0f);
         const int jb = max(sg.gb - gb8, 0), je = min(sg.ge - gb8, 8);
@@ -757,7 +759,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
       }
       // ---- segment finished: write the tile, or hand its partial to the fixup
       if (et == 0) trace_stamp(args, 15, 4 * k);
-      aborted = aborted || bar_red_or(1, NE, !ok);
+      aborted = bar_red_or(1, NE, aborted || !ok);   // every thread takes part, always
       if (aborted) break;
       if constexpr (C::TEAMS == 2 && !DUMP) {
         // the second team hands its sums to the first, which adds them (fixed order)

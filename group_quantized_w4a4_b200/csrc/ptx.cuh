@@ -171,13 +171,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* map, uint3
       : "memory");
 }
 
-// Prefetch one box of a 2-D tiled tensor map into L2 (no shared memory, no completion).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const void* map, int c0, int c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map),
-               "r"(c0), "r"(c1)
-               : "memory");
-}
-
 // Order this thread's generic-proxy shared-memory writes before later async-proxy reads
 // (tensor core operand fetches).
 __device__ __forceinline__ void fence_proxy_async_smem() {
