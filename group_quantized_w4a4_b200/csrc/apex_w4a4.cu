@@ -116,6 +116,7 @@ struct Plan {
   int S = 0;        // K-stages (pairs of groups) per tile
   int P = 0;        // persistent CTAs
   int streamk = 0;  // stream-K partition (needs workspace) or whole tiles round-robin
+  int cluster = 1;  // >1: each tile split over this many CTAs of one thread-block cluster
 };
 
 int pick_bt(int64_t M) {
@@ -152,6 +153,10 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, bool allow_streamk) {
     if ((long long)p.P * units >= (1ll << 31)) {   // the device partition math is 32-bit
       p.streamk = 0;
       p.P = p.T < sms ? p.T : sms;
+    } else if (per_tile >= 2 && per_tile <= apex::max_cluster(p.bt) && p.S >= per_tile &&
+               p.P == per_tile * p.T) {
+      // each tile's CTAs as one cluster: the parts are added in the owner's shared memory
+      p.cluster = per_tile;
     }
   }
   return p;
@@ -181,24 +186,35 @@ struct Maps {
 // Every kernel is launched as a programmatic dependent of the previous work in the stream,
 // so its launch and prologue overlap that work's tail (each kernel waits for the previous
 // grid before its first global access).
+// cluster > 1: consecutive CTAs form thread-block clusters of that size.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem,
-                       cudaStream_t s, Args... args) {
+cudaError_t launch_pdl_cl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                          cudaStream_t s, unsigned cluster, Args... args) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(block);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;
+  at[1].val.clusterDim.x = cluster;
+  at[1].val.clusterDim.y = 1;
+  at[1].val.clusterDim.z = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = cluster > 1 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                       cudaStream_t s, Args... args) {
+  return launch_pdl_cl(kern, grid, block, smem, s, 1u, args...);
+}
+
 template <int BT, int MODE>
-apex_status_t launch_bt(const Plan& p, const Maps& m, const GemmArgs& a, cudaStream_t s) {
+apex_status_t launch_bt(const Plan& p, const Maps& m, GemmArgs a, cudaStream_t s) {
   using C = GemmCfg<BT, MODE>;
   auto kern = apex::w4a4_gemm_kernel<BT, MODE>;
   static thread_local int attr_dev = -1;   // the attribute is per device; set it once each
@@ -210,7 +226,35 @@ apex_status_t launch_bt(const Plan& p, const Maps& m, const GemmArgs& a, cudaStr
       return APEX_ERR_CUDA;
     attr_dev = dev;
   }
-  return cuda_status(launch_pdl(kern, (unsigned)p.P, C::THREADS, (size_t)C::SMEM, s, m.w, m.a, a));
+  if (a.cluster > 1) {
+    // Clusters only pay when all of them are resident at once (one CTA per SM); otherwise
+    // the parts go through global memory.  The answer is cached per device and size.
+    static thread_local int occ_dev = -1, occ_size = 0, occ_clusters = 0;
+    if (occ_dev != dev || occ_size != a.cluster) {
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = dim3((unsigned)p.P);
+      cfg.blockDim = dim3(C::THREADS);
+      cfg.dynamicSmemBytes = (size_t)C::SMEM;
+      cudaLaunchAttribute at{};
+      at.id = cudaLaunchAttributeClusterDimension;
+      at.val.clusterDim.x = (unsigned)a.cluster;
+      at.val.clusterDim.y = 1;
+      at.val.clusterDim.z = 1;
+      cfg.attrs = &at;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+      }
+      occ_dev = dev;
+      occ_size = a.cluster;
+      occ_clusters = n;
+    }
+    if ((long long)occ_clusters * a.cluster < p.P) a.cluster = 1;
+  }
+  return cuda_status(launch_pdl_cl(kern, (unsigned)p.P, C::THREADS, (size_t)C::SMEM, s,
+                                   (unsigned)a.cluster, m.w, m.a, a));
 }
 
 template <int MODE>
@@ -245,6 +289,7 @@ GemmArgs base_args(const Plan& p, int64_t M, int64_t N, int64_t K, int32_t gw,
   a.TS = p.streamk ? p.T * p.S : 0;
   a.P = p.P;
   a.streamk = p.streamk;
+  a.cluster = p.cluster;
   // Scales are fetched in 16-byte blocks of 8 groups when rows are 16-byte strided.
   a.sa_vec = a.G % 8 == 0 && a_scales && aligned(a_scales, 16);
   a.sw_vec = gw == 128 && a.G % 8 == 0 && w_scales && aligned(w_scales, 16);

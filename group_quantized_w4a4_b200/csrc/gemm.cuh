@@ -64,6 +64,9 @@ struct GemmArgs {
   int TS;            // T * S
   int P;             // persistent CTAs (gridDim.x)
   int streamk;       // 1: contiguous stage ranges per CTA; 0: whole tiles round-robin
+  int cluster;       // >1: every tile is split over `cluster` consecutive CTAs launched as one
+                     // thread-block cluster, which add their parts in the owner's shared
+                     // memory (max_cluster(BT) at most); 1: parts go through global memory
   int sa_vec;        // sa rows readable as 16-byte vectors of 8 groups
   int sw_vec;        // sw rows readable as 16-byte vectors of 8 groups (gw == 128)
   const __half* sa;  // [M][G]
@@ -108,6 +111,10 @@ __device__ __forceinline__ void trace_stamp(const GemmArgs& a, int role, int ste
 // boxes of packed weights), so the per-stage hand-off costs are spread over more MMAs.
 __host__ __device__ constexpr int stage_groups(int bt) { return bt <= 32 ? 4 : 2; }
 
+// Largest cluster whose partial tiles (fp32 [BT][128] per partner) the owner CTA can take
+// in shared memory: the narrow tiles of decode-sized batches.
+__host__ __device__ constexpr int max_cluster(int bt) { return bt == 16 ? 4 : bt == 32 ? 2 : 1; }
+
 template <int BT, int MODE>
 struct GemmCfg {
   static constexpr bool AQ8 = MODE == MODE_AQ8;
@@ -141,14 +148,18 @@ struct GemmCfg {
   // token scales: per team, 2 blocks x [8 groups][BT] fp32
   static constexpr int SAT = 2 * TEAMS * 8 * BT * 4;
   static constexpr int RED = TEAMS == 2 ? CPT * BM * 4 : 0;   // second team's sums [CPT][BM]
-  static constexpr int FIXED = NX * XA + SAT + RED + 4096;
+  // partners' partial tiles, received by a cluster's owner: [partner][BM rows][BT] fp32
+  static constexpr int MAXCL = max_cluster(BT);
+  static constexpr int RCV = (MAXCL - 1) * BT * BM * 4;
+  static constexpr int FIXED = NX * XA + SAT + RED + RCV + 4096;
   static constexpr int NP_FIT = (200 * 1024 - FIXED) / PK_STAGE;
   static constexpr int NP = NP_FIT > 12 ? 12 : (NP_FIT < 2 ? 2 : NP_FIT);  // packed stages
   static constexpr int OFF_PK = 0;
   static constexpr int OFF_XA = OFF_PK + NP * PK_STAGE;
   static constexpr int OFF_SAT = OFF_XA + NX * XA;
   static constexpr int OFF_RED = OFF_SAT + SAT;
-  static constexpr int OFF_BAR = OFF_RED + RED;
+  static constexpr int OFF_RCV = OFF_RED + RED;
+  static constexpr int OFF_BAR = OFF_RCV + RCV;
   // Hand-off unit: the groups that pass between converters, MMA and epilogue under one
   // barrier phase -- a whole stage for narrow tiles (the MMA issue loop is short on work
   // per group there), a single group for wide ones (whose partial slots fill TMEM).
@@ -157,7 +168,7 @@ struct GemmCfg {
   static constexpr int NDU = NSLOT / GPB;   // partial hand-off units in flight
   static_assert(NX % GPB == 0 && NSLOT % GPB == 0, "slots come in whole units");
   static_assert(GPB == 1 || CWG * (KPS / CWG) == KPS, "converter split");
-  static constexpr int NBAR = 2 * NP + 2 * NXU + NDU + 1;
+  static constexpr int NBAR = 2 * NP + 2 * NXU + NDU + 2;
   // one MMA-completion barrier per operand unit also tells the epilogue that the unit's
   // partials are ready, which needs every partial slot to be reused no sooner than its
   // operand slot
@@ -285,6 +296,8 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
   uint64_t* g_done = x_full + C::NXU;
   uint64_t* d_empty = g_done + C::NXU;
   uint64_t* mma_done = d_empty + C::NDU;
+  uint64_t* rcv_full = mma_done + 1;   // a cluster owner: every partner's part has landed
+  float* s_rcv = reinterpret_cast<float*>(smem + C::OFF_RCV);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* s_abort = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
   int* s_last = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
@@ -311,6 +324,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
       mbar_init(smem_u32(&d_empty[i]), C::GPB == 1 ? C::EPI_WARPS : 1);
     }
     mbar_init(smem_u32(mma_done), 1);
+    mbar_init(smem_u32(rcv_full), 1);
     *s_abort = 0;
     *s_last = 0;
     *s_never = 0;
@@ -327,6 +341,12 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // A split tile's CTAs may form one cluster, whose partners write into the owner's shared
+  // memory at the end.  Announce here that this CTA's barriers are initialised; the
+  // matching wait comes before the first remote access, long after, so it costs nothing.
+  const bool clustered = C::MAXCL > 1 && !DUMP && args.cluster > 1;
+  bool cl_waited = false;   // this thread has waited for that announcement
+  if (clustered) cluster_arrive();
   // Launched as a programmatic dependent: the prologue above overlaps the previous grid's
   // tail.  The roles that touch global memory (producer, epilogue) wait for that grid
   // before their first access.
@@ -602,6 +622,9 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
     const int tt = C::TEAMS == 2 ? (et & 127) : et;
     const int M = args.M, N = args.N;
     const bool sa_vec = args.sa_vec != 0, sw_vec = args.sw_vec != 0;
+    // cluster mode: every tile is split over exactly `cluster` CTAs, the owner at rank 0
+    bool expected = false;   // an owner: the parts' byte count is armed on rcv_full
+    bool received = false;   // an owner: its partners' parts are in its shared memory
 
     // Scales of the 8-group block starting at gb8 of segment sg (this thread's token / row).
     auto block_scales = [&](const Seg& sg, int gb8, uint4& sa, uint4& sw) {
@@ -785,7 +808,40 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
         }
         const int cf = args.streamk ? sk_owner(args, sg.t * args.S) : (int)blockIdx.x;
         const int cl = args.streamk ? sk_owner(args, sg.t * args.S + args.S - 1) : (int)blockIdx.x;
-        if (cf == cl) {
+        if (clustered) {
+          // The parts meet in the owner's shared memory.  A partner sends its part after the
+          // segment loop (below), on every path; the owner takes them here, adds them in
+          // CTA order and writes the tile.
+          if (blockIdx.x % (unsigned)args.cluster == 0) {
+            if (et == 0)
+              mbar_arrive_expect_tx(smem_u32(rcv_full),
+                                    (uint32_t)((args.cluster - 1) * BT * C::BM * 4));
+            expected = true;
+            ok = mbar_wait_cluster(smem_u32(rcv_full), 0u, lim, abort_flag);
+            received = ok;
+            if (et == 0) trace_stamp(args, 15, 4 * k + 2);
+            aborted = bar_red_or(FB, NF, !ok);
+            if (aborted) break;
+            for (int c = 1; c < args.cluster; ++c) {
+              const float4* src = reinterpret_cast<const float4*>(
+                  s_rcv + ((size_t)(c - 1) * C::BM + row) * C::CPT);
+#pragma unroll
+              for (int e = 0; e < C::CPT; e += 4) {
+                const float4 v = src[e / 4];
+                acc[e / 2].x += v.x;
+                acc[e / 2].y += v.y;
+                acc[e / 2 + 1].x += v.z;
+                acc[e / 2 + 1].y += v.w;
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < C::CPT; ++e) {
+              const int m = m0 + h * 64 + e;
+              const float v = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
+              if (m < M && nvalid) args.y[(size_t)m * N + n] = __float2half_rn(v);
+            }
+          }
+        } else if (cf == cl) {
 #pragma unroll
           for (int e = 0; e < C::CPT; ++e) {
             const int m = m0 + h * 64 + e;
@@ -859,10 +915,40 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
       have = have_next;
       sg = nx;
     }
+    if (clustered && team == 0) {
+      const int cl_rank = (int)(blockIdx.x % (unsigned)args.cluster);
+      if (cl_rank != 0) {
+        // A partner's part (its one segment's sums; whatever it holds if the CTA gave up)
+        // goes to the owner on every path, so the owner's wait below always ends.
+        cluster_wait();   // the owner's barriers are initialised
+        cl_waited = true;
+        const uint32_t dst = cluster_map(
+            smem_u32(s_rcv + ((size_t)(cl_rank - 1) * C::BM + row) * C::CPT), 0u);
+        const uint32_t bar = cluster_map(smem_u32(rcv_full), 0u);
+#pragma unroll
+        for (int e = 0; e < C::CPT; e += 4)
+          st_async_v4(dst + 4u * e, acc[e / 2].x, acc[e / 2].y, acc[e / 2 + 1].x,
+                      acc[e / 2 + 1].y, bar);
+        if (et == 0) trace_stamp(args, 15, 1);
+      } else if (!received) {
+        // an owner that gave up before its flush still takes its partners' parts, so that no
+        // store into this CTA's shared memory is in flight when it exits
+        if (et == 0 && !expected)
+          mbar_arrive_expect_tx(smem_u32(rcv_full),
+                                (uint32_t)((args.cluster - 1) * BT * C::BM * 4));
+        mbar_wait_cluster(smem_u32(rcv_full), 0u, 2 * lim, never);
+      }
+    }
   }
 
   tc_fence_before();
   __syncthreads();
+  if (clustered) {
+    // no CTA of the cluster exits while stores into its shared memory may be in flight
+    if (!cl_waited) cluster_wait();
+    cluster_arrive();
+    cluster_wait();
+  }
   if (threadIdx.x == 0) trace_stamp(args, 5, 1);
   if (warp == 1) {
     tc_fence_after();

@@ -116,6 +116,63 @@ __device__ __forceinline__ bool mbar_wait2(uint32_t a, uint32_t pa, uint32_t b, 
          (rb || mbar_wait(b, pb, limit_ns, abort_flag));
 }
 
+// ------------------------------------------------------------------ thread-block clusters
+// (a CTA launched without a cluster is a cluster of one)
+
+// Cluster barrier, split: every thread of every CTA of the cluster arrives (release), and
+// later waits (acquire) for all of them; arrivals and waits alternate per thread.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// The shared::cluster address of shared variable `saddr` (a shared::cta address) in the
+// CTA of the cluster with rank `rank`.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+// Asynchronous 16-byte store into another CTA's shared memory (raddr, a shared::cluster
+// address); its bytes count towards the transaction count of that CTA's mbarrier rbar.
+__device__ __forceinline__ void st_async_v4(uint32_t raddr, float a, float b, float c, float d,
+                                            uint32_t rbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, "
+      "[%5];" ::"r"(raddr),
+      "f"(a), "f"(b), "f"(c), "f"(d), "r"(rbar)
+      : "memory");
+}
+
+// As mbar_wait, with acquire at cluster scope: for data that other CTAs of the cluster
+// wrote into this CTA's shared memory against this barrier.
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
+                                                  uint64_t limit_ns, volatile int* abort_flag) {
+  const uint64_t t0 = clock_cycles();
+  for (uint32_t spin = 0;; ++spin) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((spin & 15u) == 15u) {
+      if (*abort_flag) return false;
+      if (clock_cycles() - t0 > 2 * limit_ns || spin > (1u << 30)) {
+        atomicOr(&g_device_status, DEV_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // GPU-scope acquire-release fence.  After a CTA barrier it also orders the other threads'
 // earlier writes (cumulativity), so one thread can publish a CTA's results.
 __device__ __forceinline__ void fence_acq_rel_gpu() {
