@@ -210,6 +210,24 @@ def test_gemm_split_k_is_deterministic(apex):
     assert int(ws[:256].sum()) == 0        # arrival counters are left at zero
 
 
+@pytest.mark.parametrize("M,ways", [(16, 2), (16, 3), (16, 4), (32, 2), (5, 4)])
+def test_gemm_split_over_a_cluster_matches_oracle(apex, M, ways):
+    # N chosen so that every tile is split `ways` ways on this device (one CTA per SM):
+    # 16- and 32-token tiles split 2-4 ways run as thread-block clusters that add the parts
+    # in the owner's shared memory.  The last tile is ragged.
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    N = 128 * (sms // ways) - 50
+    K = 128 * 4 * ways * 2             # two pipeline stages per CTA
+    a = synth.activations(M, K, "outlier", 40 + ways)
+    w = synth.weights(N, K, 40 + ways)
+    ap, sa = oracle.quantize_pack(a, 128)
+    wp, sw = oracle.quantize_pack(w, 128)
+    ref = oracle.gemm(ap, sa, wp, sw, M, N, K, 128, 128)
+    y = run_gemm(apex, ap, sa, wp, sw, M, N, K, 128)
+    assert_close(y, ref)
+    assert np.array_equal(y, run_gemm(apex, ap, sa, wp, sw, M, N, K, 128))   # deterministic
+
+
 def test_gemm_scale_linearity(apex):
     M, N, K = 32, 256, 1024
     a = synth.activations(M, K, "normal", 8)
@@ -418,6 +436,30 @@ def test_pipeline_wait_timeout_is_reported_and_context_survives(apex):
     try:
         apex.apex_debug_withhold_step(1)              # one bulk copy never issued
         apex.apex_w4a4_gemm(M, N, K, 128, 128, *args, y, None)
+        assert apex.apex_get_device_status() == apex.APEX_ERR_TIMEOUT
+    finally:
+        apex.apex_set_wait_limit_ns(2_000_000_000)
+    ref = oracle.gemm(ap, sa, wp, sw, M, N, K, 128, 128)
+    assert_close(run_gemm(apex, ap, sa, wp, sw, M, N, K, 128), ref)
+
+
+def test_cluster_wait_timeout_is_reported_and_context_survives(apex):
+    # The same failure inside a clustered split: every CTA gives up at its second stage,
+    # the partners still send their parts, the owners still take them, and the launch ends.
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    M, N, K = 16, 128 * (sms // 2), 2048
+    a = synth.activations(M, K, "normal", 5)
+    w = synth.weights(N, K, 5)
+    ap, sa = oracle.quantize_pack(a, 128)
+    wp, sw = oracle.quantize_pack(w, 128)
+    args = [dev(x) for x in (ap, sa, wp, sw)]
+    y = torch.zeros((M, N), dtype=torch.float16, device="cuda")
+    ws = apex.workspace(M, N, K)
+    assert ws is not None
+    apex.apex_set_wait_limit_ns(50_000_000)           # 50 ms
+    try:
+        apex.apex_debug_withhold_step(1)              # every CTA's second stage never issued
+        apex.apex_w4a4_gemm(M, N, K, 128, 128, *args, y, ws)
         assert apex.apex_get_device_status() == apex.APEX_ERR_TIMEOUT
     finally:
         apex.apex_set_wait_limit_ns(2_000_000_000)
