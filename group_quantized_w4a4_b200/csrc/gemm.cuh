@@ -14,9 +14,14 @@
 // Persistent CTAs, one per SM, walk a list of segments (tile, K-group range):
 //   tile mode     whole tiles, round-robin over the CTAs (many tiles);
 //   stream-K      the tiles' K-stages are cut into equal contiguous ranges, one per CTA, so
-//                 every SM streams the same number of bytes (few tiles: decode, small M).
-//                 A tile covered by several CTAs is finished by the CTA holding its first
-//                 stage, which adds the others' fp32 parts in CTA order (deterministic).
+//                 every SM streams the same number of bytes (few tiles: decode, small M);
+//                 with at least two CTAs per tile, every tile is split the same number of
+//                 ways.  A tile covered by several CTAs is finished by the CTA holding its
+//                 first stage, which adds the others' fp32 parts in CTA order
+//                 (deterministic).  The parts travel through global memory (a release
+//                 counter the owner polls) or, for 16- and 32-token tiles split 2-4 ways,
+//                 inside a thread-block cluster: the partners write them into the owner's
+//                 shared memory with st.async, counted in bytes on one of its mbarriers.
 // Roles:
 //   warp 0      TMA producer: packed W tile, one [128 x 128 B] box per two K-groups (a stage
 //               holds two K-groups, four for tiles of at most 32 tokens), and
@@ -27,11 +32,12 @@
 //   warps 2..5  converters (one warpgroup): nibbles -> int8 in registers.  The weight row
 //               of each thread goes to tensor memory (tcgen05.st); packed token rows go to
 //               shared memory in the 128-byte-swizzled K-major operand layout.
-//   then        epilogue: tcgen05.ld of a group's partials while the next groups' MMAs
-//               run, fp32 scale by sa*sw and accumulate in registers (packed f32x2 math);
-//               fp16 output.  Each epilogue thread also fetches the scales it needs, one
-//               block of 8 groups ahead (its weight row's sw; one token's sa, shared with
-//               the other epilogue threads through a small transposed buffer).
+//   then        epilogue (8 warps): tcgen05.ld of a group's partials while the next
+//               groups' MMAs run, fp32 scale by sa*sw and accumulate in registers (packed
+//               f32x2 math); fp16 output.  Each epilogue thread also fetches the scales it
+//               needs, one block of 8 groups ahead (its weight row's sw; one token's sa,
+//               shared with the other threads of its team through a small transposed
+//               buffer).  Narrow tiles run two teams of 4 warps on alternate hand-off units.
 // A warp reaches tensor-memory lanes 32*(warp % 4) .. +31 only, so each group of four
 // consecutive warps covers the 128 lanes once.
 //
