@@ -315,10 +315,12 @@ apex_status_t quantize_launch(const void* x, int64_t rows, int64_t K, int32_t gr
     return APEX_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t units = rows * (K / group);
-  const int threads = 256;
+  // 128-thread blocks: one fits on an SM next to a GEMM CTA (registers), so the GEMM that
+  // follows can start its prologue on every SM while the quantizer still runs
+  const int threads = 128;
   const int64_t warps_needed = (units + 1) / 2;
   int64_t blocks = (warps_needed * 32 + threads - 1) / threads;
-  const int64_t cap = (int64_t)dev_info().sms * 16;
+  const int64_t cap = (int64_t)dev_info().sms * 32;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   const __half* xh = static_cast<const __half*>(x);
