@@ -25,7 +25,7 @@ __all__ = [
     "quantize_act_expanded",
     "apex_w4a4_gemm_workspace_size", "apex_w4a4_group_partials", "apex_get_device_status",
     "apex_set_wait_limit_ns", "apex_status_string", "apex_debug_withhold_step",
-    "apex_debug_trace_next_gemm",
+    "apex_debug_trace_next_gemm", "apex_debug_gemm_plan",
     "pack_weights", "quantize_act", "gemm", "workspace",
 ]
 
@@ -97,6 +97,8 @@ def load_library(build_if_missing: bool = True):
         lib.apex_debug_withhold_step.restype = None
         lib.apex_debug_trace_next_gemm.argtypes = [P, I32, I32]
         lib.apex_debug_trace_next_gemm.restype = None
+        lib.apex_debug_gemm_plan.argtypes = [I64, I64, I64, I32, I32, P]
+        lib.apex_debug_gemm_plan.restype = st
         _lib = lib
         return lib
 
@@ -237,6 +239,16 @@ def apex_debug_trace_next_gemm(trace, ctas: int, steps: int):
     if trace.numel() < ctas * 16 * steps:
         raise ValueError("trace buffer too small")
     load_library().apex_debug_trace_next_gemm(_ptr(trace), int(ctas), int(steps))
+
+
+def apex_debug_gemm_plan(M: int, N: int, K: int, sms: int, with_workspace: bool = True) -> dict:
+    """The work plan apex_w4a4_gemm would use on a GPU with `sms` SMs (host only)."""
+    import ctypes
+    out = (ctypes.c_int32 * 6)()
+    _check(load_library().apex_debug_gemm_plan(int(M), int(N), int(K), int(sms),
+                                               1 if with_workspace else 0, out),
+           "apex_debug_gemm_plan")
+    return dict(zip(("bt", "tiles", "stages", "ctas", "split_k", "cluster"), list(out)))
 
 
 # ------------------------------------------------------------------ tensor conveniences

@@ -128,7 +128,8 @@ int pick_bt(int64_t M) {
 
 // One persistent CTA per SM.  Whole tiles when there are at least 4 per SM (the last,
 // partial round costs little); otherwise stream-K, so every SM streams the same bytes.
-Plan make_plan(int64_t M, int64_t N, int64_t K, bool allow_streamk) {
+// sms_override > 0 plans for that many SMs instead of the current device's (plan tests).
+Plan make_plan(int64_t M, int64_t N, int64_t K, bool allow_streamk, int sms_override = 0) {
   Plan p;
   p.bt = pick_bt(M);
   p.tiles_n = (int)((N + 127) / 128);
@@ -137,7 +138,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, bool allow_streamk) {
   const int G = (int)(K / 128);
   const int kps = apex::stage_groups(p.bt);
   p.S = (G + kps - 1) / kps;
-  const int sms = dev_info().sms;
+  const int sms = sms_override > 0 ? sms_override : dev_info().sms;
   if (!allow_streamk || p.T >= 4 * sms) {
     p.streamk = 0;
     p.P = p.T < sms ? p.T : sms;
@@ -565,6 +566,22 @@ apex_status_t apex_get_device_status(void* stream) {
 }
 
 void apex_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns ? ns : 1; }
+
+apex_status_t apex_debug_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t sms,
+                                   int32_t with_workspace, int32_t *plan) {
+  if (!plan || sms <= 0) return APEX_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0 || K % 128 || M > INT32_MAX || N > INT32_MAX ||
+      K > INT32_MAX)
+    return APEX_ERR_INVALID_ARG;
+  const Plan p = make_plan(M, N, K, with_workspace != 0, sms);
+  plan[0] = p.bt;
+  plan[1] = p.T;
+  plan[2] = p.S;
+  plan[3] = p.P;
+  plan[4] = p.streamk;
+  plan[5] = p.cluster;
+  return APEX_OK;
+}
 
 void apex_debug_withhold_step(int32_t step) { t_withhold = step; }
 

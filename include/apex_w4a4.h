@@ -176,6 +176,18 @@ void apex_set_wait_limit_ns(uint64_t ns);
 const char *apex_status_string(apex_status_t status);
 
 /*
+ * Introspection: the work plan apex_w4a4_gemm would use for an M x N x K problem on a GPU
+ * with `sms` SMs (with_workspace != 0: a large enough workspace is given).  Writes
+ * plan[0..5] = { token tile BT, tiles, K-stages per tile, persistent CTAs, split-K (0/1),
+ * CTAs per cluster (1: the parts of split tiles go through global memory) }.  Host only;
+ * nothing is launched.  APEX_ERR_INVALID_ARG for a NULL plan, sms <= 0 or a bad shape.
+ * The launch itself may still fall back from clusters to global memory when the clusters
+ * would not all be resident at once on the actual device.
+ */
+apex_status_t apex_debug_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t sms,
+                                   int32_t with_workspace, int32_t *plan);
+
+/*
  * Test hook: the next GEMM launch on this host thread skips the bulk copy of pipeline stage
  * `step` (two or four K-groups, counted within each CTA), so its consumers wait until the
  * time limit.  -1 turns it off.  Used only to test the timeout path; never needed by callers.
@@ -192,8 +204,9 @@ void apex_debug_withhold_step(int32_t step);
  * epilogue inputs of K-group i ready, [c][8][i] MMA waits returned, [c][9][i] MMAs of
  * K-group i issued before their commits, [c][10][i] MMA wait for the operands of K-group i
  * returned, [c][11 + w][s] converter warp w (0..3 within its warpgroup) done with stage s,
- * [c][15][4k .. 4k+3] the epilogue's k-th segment: finished, partial published, arrival
- * counted, tile written;
+ * [c][15][4k .. 4k+3] the epilogue's k-th segment: finished, partial published (global
+ * hand-off; [c][15][1] is also a cluster partner's send), parts received by the owner, tile
+ * written;
  * [c][5][0] / [c][5][1] %globaltimer (ns) at CTA start / end, [c][5][2] the SM it ran on,
  * [c][5][3] clock64 at CTA start, [c][5][4] / [c][5][5] clock64 when the producer enters its
  * loop / has its first work item, [c][5][6] %globaltimer at kernel entry (before the
