@@ -395,12 +395,20 @@ def roofline_obj(g, gemm_ms_avg, peaks, peaks_kind, traffic=None):
             "kernel_ms": round(gemm_ms_avg, 5)}
 
 
-def cpu_baseline(g: synth.Gemm, budget_s: float = 20.0):
-    """The oracle, as it stands, on this host's cores: quantize the activations and run the
-    fp64 GEMM over a bounded sample of output rows; effective TOPS scaled to the rows."""
+def oracle_inputs(g: synth.Gemm):
+    """The workload's activations and the oracle's packed weights (set up once)."""
     import oracle
     a, w = synth.make(g)
     wp, sw = oracle.quantize_pack(w, g.gw)
+    return a, wp, sw
+
+
+def cpu_baseline(g: synth.Gemm, budget_s: float = 20.0, repeat_small: bool = True,
+                 inputs=None):
+    """The oracle, as it stands, on this host's cores: quantize the activations and run the
+    fp64 GEMM over a bounded sample of output rows; effective TOPS scaled to the rows."""
+    import oracle
+    a, wp, sw = inputs if inputs is not None else oracle_inputs(g)
     rows = np.arange(min(g.M, 4), dtype=np.int64)
     t0 = time.perf_counter()
     ap, sa = oracle.quantize_pack(a[rows], 128)
@@ -417,7 +425,7 @@ def cpu_baseline(g: synth.Gemm, budget_s: float = 20.0):
         dt = time.perf_counter() - t0
     # a whole small workload is repeated until about half the budget of CPU work is timed
     reps = 1
-    if n == g.M and dt < budget_s / 2:
+    if repeat_small and n == g.M and dt < budget_s / 2:
         reps = max(1, int(np.ceil((budget_s / 2) / max(dt, 1e-3))))
         t0 = time.perf_counter()
         for _ in range(reps):
@@ -544,11 +552,14 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     g = synth.workloads()[args.workload]
+    # each step a bounded sample, sized so that the whole run stays near two minutes
+    per_step = max(0.02, 120.0 / (args.steps + args.warmup))
+    inputs = oracle_inputs(g)
     vals = []
     for _ in range(args.warmup):
-        cpu_baseline(g, budget_s=4.0)
+        cpu_baseline(g, budget_s=per_step, repeat_small=False, inputs=inputs)
     for _ in range(args.steps):
-        vals.append(cpu_baseline(g, budget_s=8.0))
+        vals.append(cpu_baseline(g, budget_s=per_step, repeat_small=False, inputs=inputs))
     v = statistics.median([x["value"] for x in vals])
     cb = dict(vals[-1])
     cb["value"] = v
