@@ -210,7 +210,9 @@ void apex_debug_withhold_step(int32_t step);
  * [c][5][0] / [c][5][1] %globaltimer (ns) at CTA start / end, [c][5][2] the SM it ran on,
  * [c][5][3] clock64 at CTA start, [c][5][4] / [c][5][5] clock64 when the producer enters its
  * loop / has its first work item, [c][5][6] %globaltimer at kernel entry (before the
- * prologue).  Steps beyond `steps` are not recorded.
+ * prologue).  Steps beyond `steps` are not recorded.  clock64 counts cycles of the SM clock
+ * the kernel ran at (below the nominal maximum under load), so convert those stamps with
+ * that clock, or compare them only with each other, not with the %globaltimer ones.
  */
 void apex_debug_trace_next_gemm(uint64_t *trace, int32_t ctas, int32_t steps);
 
