@@ -22,6 +22,7 @@ __all__ = [
     "ApexError", "load_library", "library_path",
     "apex_pack_weights_int4", "apex_quantize_act_int4", "apex_w4a4_gemm",
     "apex_w4a4_gemm_noalloc", "apex_quantize_act_int4_expanded", "apex_w4a4_gemm_expanded",
+    "apex_w4a4_gemm_quant", "apex_w4a4_gemm_expanded_quant",
     "quantize_act_expanded",
     "apex_w4a4_gemm_workspace_size", "apex_w4a4_group_partials", "apex_get_device_status",
     "apex_set_wait_limit_ns", "apex_status_string", "apex_debug_withhold_step",
@@ -77,6 +78,10 @@ def load_library(build_if_missing: bool = True):
         lib.apex_w4a4_gemm_expanded.restype = st
         lib.apex_w4a4_gemm.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P, SZ, P]
         lib.apex_w4a4_gemm.restype = st
+        for name in ("apex_w4a4_gemm_quant", "apex_w4a4_gemm_expanded_quant"):
+            fn = getattr(lib, name)
+            fn.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P, P, I32, P, SZ, P]
+            fn.restype = st
         lib.apex_w4a4_gemm_noalloc.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P]
         lib.apex_w4a4_gemm_noalloc.restype = st
         lib.apex_w4a4_gemm_workspace_size.argtypes = [I64, I64, I64, I32, I32]
@@ -164,6 +169,36 @@ def apex_quantize_act_int4_expanded(x_f16, M, K, group_a, x_q8, x_scales_f16, st
                                                           _ptr(x_q8), _ptr(x_scales_f16),
                                                           _stream(stream)),
            "apex_quantize_act_int4_expanded")
+
+
+def _gemm_quant(name, M, N, K, group_a, group_w, a, a_scales, w_packed, w_scales, y_f16,
+                yq, yq_scales, yq_expanded, workspace, workspace_bytes, stream):
+    if workspace is not None and workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(getattr(load_library(), name)(M, N, K, group_a, group_w, _ptr(a), _ptr(a_scales),
+                                         _ptr(w_packed), _ptr(w_scales), _ptr(y_f16),
+                                         _ptr(yq), _ptr(yq_scales), 1 if yq_expanded else 0,
+                                         _ptr(workspace), workspace_bytes or 0,
+                                         _stream(stream)), name)
+
+
+def apex_w4a4_gemm_quant(M, N, K, group_a, group_w, a_packed, a_scales, w_packed, w_scales,
+                         y_f16, yq, yq_scales, yq_expanded=False, workspace=None,
+                         workspace_bytes=None, stream=None):
+    """The GEMM plus its output quantized as the next layer's activations (y_f16 may be
+    None); see the C header."""
+    _gemm_quant("apex_w4a4_gemm_quant", M, N, K, group_a, group_w, a_packed, a_scales,
+                w_packed, w_scales, y_f16, yq, yq_scales, yq_expanded, workspace,
+                workspace_bytes, stream)
+
+
+def apex_w4a4_gemm_expanded_quant(M, N, K, group_a, group_w, a_q8, a_scales, w_packed,
+                                  w_scales, y_f16, yq, yq_scales, yq_expanded=False,
+                                  workspace=None, workspace_bytes=None, stream=None):
+    """As apex_w4a4_gemm_quant, reading expanded activations."""
+    _gemm_quant("apex_w4a4_gemm_expanded_quant", M, N, K, group_a, group_w, a_q8, a_scales,
+                w_packed, w_scales, y_f16, yq, yq_scales, yq_expanded, workspace,
+                workspace_bytes, stream)
 
 
 def apex_w4a4_gemm_expanded(M, N, K, group_a, group_w, a_q8, a_scales, w_packed, w_scales,

@@ -214,10 +214,10 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, si
   return launch_pdl_cl(kern, grid, block, smem, s, 1u, args...);
 }
 
-template <int BT, int MODE>
+template <int BT, int MODE, bool QOUT>
 apex_status_t launch_bt(const Plan& p, const Maps& m, GemmArgs a, cudaStream_t s) {
   using C = GemmCfg<BT, MODE>;
-  auto kern = apex::w4a4_gemm_kernel<BT, MODE>;
+  auto kern = apex::w4a4_gemm_kernel<BT, MODE, QOUT>;
   static thread_local int attr_dev = -1;   // the attribute is per device; set it once each
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return APEX_ERR_CUDA;
@@ -258,14 +258,23 @@ apex_status_t launch_bt(const Plan& p, const Maps& m, GemmArgs a, cudaStream_t s
                                    (unsigned)a.cluster, m.w, m.a, a));
 }
 
+template <int MODE, bool QOUT>
+apex_status_t launch_gemm_q(const Plan& p, const Maps& m, const GemmArgs& a, cudaStream_t s) {
+  switch (p.bt) {
+    case 16: return launch_bt<16, MODE, QOUT>(p, m, a, s);
+    case 32: return launch_bt<32, MODE, QOUT>(p, m, a, s);
+    case 64: return launch_bt<64, MODE, QOUT>(p, m, a, s);
+    default: return launch_bt<128, MODE, QOUT>(p, m, a, s);
+  }
+}
+
+// The kernel with the quantized output when the arguments ask for one.
 template <int MODE>
 apex_status_t launch_gemm(const Plan& p, const Maps& m, const GemmArgs& a, cudaStream_t s) {
-  switch (p.bt) {
-    case 16: return launch_bt<16, MODE>(p, m, a, s);
-    case 32: return launch_bt<32, MODE>(p, m, a, s);
-    case 64: return launch_bt<64, MODE>(p, m, a, s);
-    default: return launch_bt<128, MODE>(p, m, a, s);
+  if constexpr (MODE != apex::MODE_DUMP) {
+    if (a.qout != nullptr) return launch_gemm_q<MODE, true>(p, m, a, s);
   }
+  return launch_gemm_q<MODE, false>(p, m, a, s);
 }
 
 // Fills the fields every mode shares.
@@ -357,6 +366,58 @@ size_t linear_act_bytes(int64_t M, int64_t K) {   // quantized activations + the
   return a + sc;
 }
 
+// The quantized output of a GEMM (all null: none).
+struct QuantOut {
+  void* q = nullptr;        // packed [M][N/2] or expanded [M][N]
+  void* scales = nullptr;   // fp16 [M][N/128]
+  bool expanded = false;
+};
+
+// Everything apex_w4a4_gemm and its variants share: argument checks, plan, launch.
+// y may be null when a quantized output is requested.
+apex_status_t gemm_entry(bool a_expanded, int64_t M, int64_t N, int64_t K, int32_t group_a,
+                         int32_t group_w, const void* a_q, const void* a_scales,
+                         const void* w_packed, const void* w_scales, void* y_f16,
+                         const QuantOut& qo, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  apex_status_t st = check_gemm_args(M, N, K, group_a, group_w);
+  if (st != APEX_OK) return st;
+  if (!a_q || !a_scales || !w_packed || !w_scales) return APEX_ERR_INVALID_ARG;
+  if (!y_f16 && !qo.q) return APEX_ERR_INVALID_ARG;
+  if (qo.q && !qo.scales) return APEX_ERR_INVALID_ARG;
+  if (qo.q && N % 128) return APEX_ERR_UNSUPPORTED;   // the output's groups are whole tiles
+  if (!aligned(a_q, 16) || !aligned(w_packed, 16) || !aligned(a_scales, 2) ||
+      !aligned(w_scales, 2) || (y_f16 && !aligned(y_f16, 2)) ||
+      (qo.q && (!aligned(qo.q, 4) || !aligned(qo.scales, 2))) ||
+      (workspace && !aligned(workspace, 256)))
+    return APEX_ERR_ALIGNMENT;
+
+  Plan p = make_plan(M, N, K, true);
+  // Without a large enough workspace, whole tiles only.
+  if (p.streamk && (!workspace || workspace_for(p) > workspace_bytes)) p = make_plan(M, N, K, false);
+  GemmArgs a = base_args(p, M, N, K, group_w, a_scales, w_scales, y_f16);
+  a.qout = static_cast<uint8_t*>(qo.q);
+  a.qscale = static_cast<__half*>(qo.scales);
+  a.qexp = qo.expanded ? 1 : 0;
+  attach_workspace(p, a, workspace);
+  a.withhold = t_withhold;
+  t_withhold = -1;
+  a.trace = t_trace;
+  a.trace_ctas = t_trace_ctas;
+  a.trace_steps = t_trace_steps;
+  t_trace = nullptr;
+
+  Maps maps;
+  memset(&maps, 0, sizeof(maps));
+  if (!make_packed_map(&maps.w, w_packed, N, K, 128)) return APEX_ERR_CUDA;
+  if (a_expanded ? !make_expanded_map(&maps.a, a_q, M, K, p.bt)
+                 : !make_packed_map(&maps.a, a_q, M, K, p.bt))
+    return APEX_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return a_expanded ? launch_gemm<apex::MODE_AQ8>(p, maps, a, s)
+                    : launch_gemm<apex::MODE_PACKED>(p, maps, a, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -381,26 +442,39 @@ apex_status_t apex_w4a4_gemm_expanded(int64_t M, int64_t N, int64_t K, int32_t g
                                       int32_t group_w, const void* a_q8, const void* a_scales,
                                       const void* w_packed, const void* w_scales, void* y_f16,
                                       void* workspace, size_t workspace_bytes, void* stream) {
-  apex_status_t st = check_gemm_args(M, N, K, group_a, group_w);
-  if (st != APEX_OK) return st;
-  if (!a_q8 || !a_scales || !w_packed || !w_scales || !y_f16) return APEX_ERR_INVALID_ARG;
-  if (!aligned(a_q8, 16) || !aligned(w_packed, 16) || !aligned(a_scales, 2) ||
-      !aligned(w_scales, 2) || !aligned(y_f16, 2) || (workspace && !aligned(workspace, 256)))
-    return APEX_ERR_ALIGNMENT;
-  Plan p = make_plan(M, N, K, true);
-  if (p.streamk && (!workspace || workspace_for(p) > workspace_bytes)) p = make_plan(M, N, K, false);
-  GemmArgs a = base_args(p, M, N, K, group_w, a_scales, w_scales, y_f16);
-  attach_workspace(p, a, workspace);
-  a.trace = t_trace;
-  a.trace_ctas = t_trace_ctas;
-  a.trace_steps = t_trace_steps;
-  t_trace = nullptr;
-  Maps maps;
-  memset(&maps, 0, sizeof(maps));
-  if (!make_packed_map(&maps.w, w_packed, N, K, 128) ||
-      !make_expanded_map(&maps.a, a_q8, M, K, p.bt))
-    return APEX_ERR_CUDA;
-  return launch_gemm<apex::MODE_AQ8>(p, maps, a, static_cast<cudaStream_t>(stream));
+  if (!y_f16) return APEX_ERR_INVALID_ARG;
+  return gemm_entry(true, M, N, K, group_a, group_w, a_q8, a_scales, w_packed, w_scales, y_f16,
+                    QuantOut{}, workspace, workspace_bytes, stream);
+}
+
+apex_status_t apex_w4a4_gemm_quant(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                   int32_t group_w, const void* a_packed, const void* a_scales,
+                                   const void* w_packed, const void* w_scales, void* y_f16,
+                                   void* yq, void* yq_scales, int32_t yq_expanded,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  QuantOut qo;
+  qo.q = yq;
+  qo.scales = yq_scales;
+  qo.expanded = yq_expanded != 0;
+  if (!yq) return APEX_ERR_INVALID_ARG;
+  return gemm_entry(false, M, N, K, group_a, group_w, a_packed, a_scales, w_packed, w_scales,
+                    y_f16, qo, workspace, workspace_bytes, stream);
+}
+
+apex_status_t apex_w4a4_gemm_expanded_quant(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                            int32_t group_w, const void* a_q8,
+                                            const void* a_scales, const void* w_packed,
+                                            const void* w_scales, void* y_f16, void* yq,
+                                            void* yq_scales, int32_t yq_expanded,
+                                            void* workspace, size_t workspace_bytes,
+                                            void* stream) {
+  QuantOut qo;
+  qo.q = yq;
+  qo.scales = yq_scales;
+  qo.expanded = yq_expanded != 0;
+  if (!yq) return APEX_ERR_INVALID_ARG;
+  return gemm_entry(true, M, N, K, group_a, group_w, a_q8, a_scales, w_packed, w_scales, y_f16,
+                    qo, workspace, workspace_bytes, stream);
 }
 
 size_t apex_w4a4_linear_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group_a,
@@ -444,31 +518,9 @@ apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, i
                              const void* a_packed, const void* a_scales, const void* w_packed,
                              const void* w_scales, void* y_f16, void* workspace,
                              size_t workspace_bytes, void* stream) {
-  apex_status_t st = check_gemm_args(M, N, K, group_a, group_w);
-  if (st != APEX_OK) return st;
-  if (!a_packed || !a_scales || !w_packed || !w_scales || !y_f16) return APEX_ERR_INVALID_ARG;
-  if (!aligned(a_packed, 16) || !aligned(w_packed, 16) || !aligned(a_scales, 2) ||
-      !aligned(w_scales, 2) || !aligned(y_f16, 2) || (workspace && !aligned(workspace, 256)))
-    return APEX_ERR_ALIGNMENT;
-
-  Plan p = make_plan(M, N, K, true);
-  // Without a large enough workspace, whole tiles only.
-  if (p.streamk && (!workspace || workspace_for(p) > workspace_bytes)) p = make_plan(M, N, K, false);
-  GemmArgs a = base_args(p, M, N, K, group_w, a_scales, w_scales, y_f16);
-  attach_workspace(p, a, workspace);
-  a.withhold = t_withhold;
-  t_withhold = -1;
-  a.trace = t_trace;
-  a.trace_ctas = t_trace_ctas;
-  a.trace_steps = t_trace_steps;
-  t_trace = nullptr;
-
-  Maps maps;
-  memset(&maps, 0, sizeof(maps));
-  if (!make_packed_map(&maps.w, w_packed, N, K, 128) ||
-      !make_packed_map(&maps.a, a_packed, M, K, p.bt))
-    return APEX_ERR_CUDA;
-  return launch_gemm<apex::MODE_PACKED>(p, maps, a, static_cast<cudaStream_t>(stream));
+  if (!y_f16) return APEX_ERR_INVALID_ARG;
+  return gemm_entry(false, M, N, K, group_a, group_w, a_packed, a_scales, w_packed, w_scales,
+                    y_f16, QuantOut{}, workspace, workspace_bytes, stream);
 }
 
 // ------------------------------------------------------------------ allocation-free GEMM

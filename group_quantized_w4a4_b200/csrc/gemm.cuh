@@ -53,6 +53,7 @@
 #include <stdint.h>
 
 #include "ptx.cuh"
+#include "quantize.cuh"
 
 namespace apex {
 
@@ -77,7 +78,13 @@ struct GemmArgs {
   int sw_vec;        // sw rows readable as 16-byte vectors of 8 groups (gw == 128)
   const __half* sa;  // [M][G]
   const __half* sw;  // [N][Gw]
-  __half* y;         // [M][N]
+  __half* y;         // [M][N], or null when only the quantized output is wanted
+  // Optional quantized output (null: none): Y's fp16 values quantized as the next layer's
+  // activations, one scale per token per 128 outputs (N % 128 == 0).  qexp 0: packed
+  // nibbles [M][N/2]; 1: the expanded operand form [M][N] (16*q bytes, GEMM K order).
+  uint8_t* qout;
+  __half* qscale;    // [M][N/128]
+  int qexp;
   float* part;       // stream-K partial tiles [P][BT][128] fp32 (one per CTA)
   unsigned* counters;  // [T] arrival counters of split tiles (zero between calls)
   int32_t* dump;     // [G][M][N] per-group partials (debug kernel only)
@@ -279,7 +286,9 @@ __device__ __forceinline__ bool get_seg(const GemmArgs& a, int k, Seg& sg) {
   return true;
 }
 
-template <int BT, int MODE>
+// QOUT: the quantized output (args.qout) is written; a separate instantiation, so plain
+// GEMMs carry none of its code.
+template <int BT, int MODE, bool QOUT = false>
 __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmW,
                      const __grid_constant__ CUtensorMap tmA, const GemmArgs args) {
@@ -647,6 +656,76 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
     };
 
     float2 acc[C::CPT / 2];
+    // Where the finished tile is written: from one call site after the hand-off (always with
+    // the quantized output; for 128-token tiles also without it, measured 2-3 % faster), or
+    // in place at each hand-off path (narrow tiles: measured faster)
+    constexpr bool ONE_WRITE = QOUT || BT >= 128;
+
+    // The finished tile goes out as fp16 Y (when args.y is set) and, when args.qout is set,
+    // as the next layer's quantized activations: for each token, the tile's 128 rows are
+    // exactly one 128-wide K-group of that token's input to the next layer, so the group's
+    // scale and codes are made here, from the fp16 values Y holds and with the rule of the
+    // activation quantizer.  Every flushing thread calls it (NF threads, barrier FB).
+    auto write_tile = [&](int m0t, int n0t) {
+      const int n = n0t + row;
+      if (args.y != nullptr) {
+#pragma unroll
+        for (int e = 0; e < C::CPT; ++e) {
+          const int m = m0t + h * C::CPT + e;
+          const float v = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
+          if (m < M && n < N) args.y[(size_t)m * N + n] = __float2half_rn(v);
+        }
+      }
+      if constexpr (!QOUT) return;
+      // each token's absmax over the tile's 128 rows: a warp's 32 rows by shuffles, then
+      // the four warps of this column block through shared memory (the first token-scale
+      // buffer of this team, idle between segments)
+      float* qmax = s_sat + h * 4 * C::CPT;   // [lane quarter][CPT]
+      const int w4 = warp & 3;
+#pragma unroll
+      for (int e = 0; e < C::CPT; ++e) {
+        const float v = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
+        float am = fabsf(__half2float(__float2half_rn(v)));
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1)
+          am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+        if (lane == 0) qmax[w4 * C::CPT + e] = am;
+      }
+      named_bar_sync(FB, NF);
+      const int kk = n0t + 32 * w4 + lane;   // this row's K index in the next layer
+#pragma unroll
+      for (int e = 0; e < C::CPT; ++e) {
+        const int m = m0t + h * C::CPT + e;
+        const float am = fmaxf(fmaxf(qmax[e], qmax[C::CPT + e]),
+                               fmaxf(qmax[2 * C::CPT + e], qmax[3 * C::CPT + e]));
+        const __half sc = group_scale(am);
+        const float v = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
+        const int qv = quant1(__half2float(__float2half_rn(v)), __half2float(sc));
+        // one byte per lane (packed: the even lanes hold k and k+1), then four bytes per word
+        uint32_t b;
+        if (args.qexp) {
+          b = ((uint32_t)qv & 15u) << 4;
+        } else {
+          const int qn = __shfl_down_sync(0xffffffffu, qv, 1);
+          b = ((uint32_t)qv & 15u) | (((uint32_t)qn & 15u) << 4);
+        }
+        const uint32_t wd = b | (__shfl_down_sync(0xffffffffu, b, 2) << 8) |
+                            (__shfl_down_sync(0xffffffffu, b, 4) << 16) |
+                            (__shfl_down_sync(0xffffffffu, b, 6) << 24);
+        if (m < M) {
+          if (args.qexp) {
+            // lane 8c: k = 8c, 8c+2, 8c+4, 8c+6 of the chunk; lane 8c+1: the odd k
+            if ((lane & 7) < 2)
+              *reinterpret_cast<uint32_t*>(args.qout + (size_t)m * N + (kk & ~7) +
+                                           4 * (lane & 1)) = wd;
+          } else if ((lane & 7) == 0) {
+            *reinterpret_cast<uint32_t*>(args.qout + (size_t)m * (N / 2) + kk / 2) = wd;
+          }
+          if (w4 == 0 && lane == 0) args.qscale[(size_t)m * (N / 128) + n0t / 128] = sc;
+        }
+      }
+      named_bar_sync(FB, NF);   // qmax is free again
+    };
     // Narrow tiles pipeline the partial loads within a hand-off unit.
     constexpr bool PIPE = C::CPT == 16 && C::GPB > 1;
     bool ok = true, aborted = false;
@@ -814,6 +893,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
         }
         const int cf = args.streamk ? sk_owner(args, sg.t * args.S) : (int)blockIdx.x;
         const int cl = args.streamk ? sk_owner(args, sg.t * args.S + args.S - 1) : (int)blockIdx.x;
+        bool owner_done = false;   // this CTA holds the whole tile now: write it
         if (clustered) {
           // The parts meet in the owner's shared memory.  A partner sends its part after the
           // segment loop (below), on every path; the owner takes them here, adds them in
@@ -840,19 +920,27 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
                 acc[e / 2 + 1].y += v.w;
               }
             }
+            if constexpr (ONE_WRITE) {
+              owner_done = true;
+            } else {
 #pragma unroll
-            for (int e = 0; e < C::CPT; ++e) {
-              const int m = m0 + h * 64 + e;
-              const float v = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
-              if (m < M && nvalid) args.y[(size_t)m * N + n] = __float2half_rn(v);
+              for (int e = 0; e < C::CPT; ++e) {
+                const int m = m0 + h * C::CPT + e;
+                const float v = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
+                if (m < M && nvalid) args.y[(size_t)m * N + n] = __float2half_rn(v);
+              }
             }
           }
         } else if (cf == cl) {
+          if constexpr (ONE_WRITE) {
+            owner_done = true;
+          } else {
 #pragma unroll
-          for (int e = 0; e < C::CPT; ++e) {
-            const int m = m0 + h * 64 + e;
-            const float v = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
-            if (m < M && nvalid) args.y[(size_t)m * N + n] = __float2half_rn(v);
+            for (int e = 0; e < C::CPT; ++e) {
+              const int m = m0 + h * C::CPT + e;
+              const float v = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
+              if (m < M && nvalid) args.y[(size_t)m * N + n] = __float2half_rn(v);
+            }
           }
         } else {
           // A split tile is finished by its owner, the CTA holding the tile's first stage:
@@ -907,14 +995,21 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
                   }
               }
             }
+            if constexpr (ONE_WRITE) {
+              owner_done = true;
+            } else {
 #pragma unroll
-            for (int e = 0; e < C::CPT; ++e) {
-              const int m = m0 + h * 64 + e;
-              const float val = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
-              if (m < M && nvalid) args.y[(size_t)m * N + n] = __float2half_rn(val);
+              for (int e = 0; e < C::CPT; ++e) {
+                const int m = m0 + h * C::CPT + e;
+                const float v = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
+                if (m < M && nvalid) args.y[(size_t)m * N + n] = __float2half_rn(v);
+              }
             }
             if (et == 0) args.counters[sg.t] = 0u;   // nobody else touches it in this launch
           }
+        }
+        if constexpr (ONE_WRITE) {
+          if (owner_done) write_tile(m0, n0);   // the whole team takes it together
         }
       }
       if (et == 0) trace_stamp(args, 15, 4 * k + 3);

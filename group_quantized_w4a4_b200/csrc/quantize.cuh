@@ -34,21 +34,23 @@ __device__ __forceinline__ __half group_scale(float absmax) {
   return __float2half_rn(__fdiv_rn(absmax, 7.0f));
 }
 
-// Quantize 8 fp16 values against scale sf (fp32 copy of the stored fp16 scale) and pack
-// them into 4 bytes (little-endian: element 0 in the low nibble of byte 0).
+// One value (an fp16 value widened to fp32) against scale sf (fp32 copy of the stored fp16
+// scale): clamp(round_half_even(f / sf), -8, 7), 0 when sf == 0.
+__device__ __forceinline__ int quant1(float f, float sf) {
+  if (sf == 0.0f) return 0;
+  const int q = __float2int_rn(__fdiv_rn(f, sf));
+  return min(max(q, -8), 7);
+}
+
+// Quantize 8 fp16 values against scale sf and pack them into 4 bytes (little-endian:
+// element 0 in the low nibble of byte 0).
 __device__ __forceinline__ uint32_t quant_pack8(const uint4& v, float sf) {
   const __half2* h = reinterpret_cast<const __half2*>(&v);
   uint32_t out = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    float2 f = __half22float2(h[i]);
-    int q0 = 0, q1 = 0;
-    if (sf != 0.0f) {
-      q0 = __float2int_rn(__fdiv_rn(f.x, sf));
-      q1 = __float2int_rn(__fdiv_rn(f.y, sf));
-      q0 = min(max(q0, -8), 7);
-      q1 = min(max(q1, -8), 7);
-    }
+    const float2 f = __half22float2(h[i]);
+    const int q0 = quant1(f.x, sf), q1 = quant1(f.y, sf);
     out |= ((uint32_t)(q0 & 0xF) | ((uint32_t)(q1 & 0xF) << 4)) << (8 * i);
   }
   return out;

@@ -105,6 +105,33 @@ apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, i
                              size_t workspace_bytes, void *stream);
 
 /*
+ * The W4A4 GEMM whose output is also quantized as the next layer's activations (a chain of
+ * W4A4 layers without a separate quantizer pass): the same computation and rules as
+ * apex_w4a4_gemm, and additionally
+ *   yq [M][N/2] packed int4 (yq_expanded == 0) or [M][N] 16*q bytes in the GEMM's
+ *      expanded operand order (yq_expanded != 0), with yq_scales [M][N/128] fp16:
+ * exactly what apex_quantize_act_int4 (or _expanded) would make, with group_a = 128, from
+ * the fp16 Y this call computes -- every tile of 128 outputs is one K-group of the next
+ * layer, so its scale and codes are made in the GEMM's epilogue.
+ *   y_f16 may be NULL (then only yq and yq_scales are written).  Requires N % 128 == 0
+ *   (APEX_ERR_UNSUPPORTED otherwise); yq 4-byte and yq_scales 2-byte aligned.
+ */
+apex_status_t apex_w4a4_gemm_quant(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                   int32_t group_w, const void *a_packed, const void *a_scales,
+                                   const void *w_packed, const void *w_scales, void *y_f16,
+                                   void *yq, void *yq_scales, int32_t yq_expanded,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* As apex_w4a4_gemm_quant, reading expanded activations (see apex_w4a4_gemm_expanded). */
+apex_status_t apex_w4a4_gemm_expanded_quant(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                            int32_t group_w, const void *a_q8,
+                                            const void *a_scales, const void *w_packed,
+                                            const void *w_scales, void *y_f16, void *yq,
+                                            void *yq_scales, int32_t yq_expanded,
+                                            void *workspace, size_t workspace_bytes,
+                                            void *stream);
+
+/*
  * Allocation-free variant of apex_w4a4_gemm.  The paper has no counterpart: this entry
  * point exists for callers that cannot allocate device memory while they run -- serving
  * runtimes that budget every device byte up front and hand out no scratch, plugin hosts

@@ -465,3 +465,94 @@ def test_cluster_wait_timeout_is_reported_and_context_survives(apex):
         apex.apex_set_wait_limit_ns(2_000_000_000)
     ref = oracle.gemm(ap, sa, wp, sw, M, N, K, 128, 128)
     assert_close(run_gemm(apex, ap, sa, wp, sw, M, N, K, 128), ref)
+
+
+# ------------------------------------------------------------------ quantized output
+
+
+QUANT_OUT_SHAPES = [
+    (16, 9472, 1024),    # 74 tiles: 2-CTA clusters on a B200
+    (16, 1024, 1024),    # split through global memory
+    (16, 256, 512),      # whole tiles
+    (1, 384, 1024),
+    (17, 2048, 1024),    # 32-token tiles, split through global memory
+    (64, 1024, 512),
+    (100, 512, 768),
+    (200, 384, 1024),    # 128-token tiles, ragged token block
+]
+
+
+@pytest.mark.parametrize("M,N,K", QUANT_OUT_SHAPES)
+@pytest.mark.parametrize("expanded_in", [False, True])
+@pytest.mark.parametrize("expanded_out", [False, True])
+def test_gemm_quantized_output_is_the_quantizer_of_y(apex, M, N, K, expanded_in, expanded_out):
+    """The fused output equals the oracle's activation quantizer applied to the fp16 Y the
+    same call wrote (bit-exact), and Y itself meets the GEMM bar."""
+    x = synth.activations(M, K, "outlier", 90 + M)
+    w = synth.weights(N, K, 90 + N)
+    ap, sa = oracle.quantize_pack(x, 128)
+    wp, sw = oracle.quantize_pack(w, 128)
+    if expanded_in:
+        a_q, a_s = apex.quantize_act_expanded(dev(x), 128)
+        fn = apex.apex_w4a4_gemm_expanded_quant
+    else:
+        a_q, a_s = dev(ap), dev(sa)
+        fn = apex.apex_w4a4_gemm_quant
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    yq = torch.empty((M, N if expanded_out else N // 2), dtype=torch.uint8, device="cuda")
+    ys = torch.empty((M, N // 128), dtype=torch.float16, device="cuda")
+    ws = apex.workspace(M, N, K)
+    fn(M, N, K, 128, 128, a_q, a_s, dev(wp), dev(sw), y, yq, ys, expanded_out, ws)
+    torch.cuda.synchronize()
+    check_status(apex)
+    y_h = host(y)
+    assert_close(y_h.astype(np.float64), oracle.gemm(ap, sa, wp, sw, M, N, K, 128, 128))
+    q_ref, s_ref = oracle.quantize_pack(y_h, 128)
+    if expanded_out:
+        assert np.array_equal(host(yq), expected_expanded(oracle.unpack(q_ref, N).astype(np.int64)))
+    else:
+        assert np.array_equal(host(yq), q_ref)
+    assert np.array_equal(f16(ys), s_ref.view(np.uint16))
+    # without Y: the same quantized output
+    yq2, ys2 = torch.zeros_like(yq), torch.zeros_like(ys)
+    fn(M, N, K, 128, 128, a_q, a_s, dev(wp), dev(sw), None, yq2, ys2, expanded_out, ws)
+    torch.cuda.synchronize()
+    check_status(apex)
+    assert torch.equal(yq2, yq) and torch.equal(ys2, ys)
+
+
+def test_gemm_quantized_output_argument_rules(apex):
+    M, N, K = 16, 200, 256                 # N not a multiple of 128
+    a = torch.zeros((M, K // 2), dtype=torch.uint8, device="cuda")
+    s = torch.zeros((M, K // 128), dtype=torch.float16, device="cuda")
+    wq = torch.zeros((N, K // 2), dtype=torch.uint8, device="cuda")
+    wsc = torch.zeros((N, K // 128), dtype=torch.float16, device="cuda")
+    yq = torch.zeros((M, N), dtype=torch.uint8, device="cuda")
+    ys = torch.zeros((M, 2), dtype=torch.float16, device="cuda")
+    with pytest.raises(apex.ApexError) as e:
+        apex.apex_w4a4_gemm_quant(M, N, K, 128, 128, a, s, wq, wsc, None, yq, ys)
+    assert e.value.code == apex.APEX_ERR_UNSUPPORTED
+    with pytest.raises(apex.ApexError) as e:
+        apex.apex_w4a4_gemm_quant(M, 256, K, 128, 128, a, s, wq, wsc, None, None, ys)
+    assert e.value.code == apex.APEX_ERR_INVALID_ARG
+
+
+def test_chained_layers_through_the_quantized_output(apex):
+    """Two W4A4 layers, the first one's quantized output fed straight to the second: the
+    second's result equals the oracle GEMM on the operands the first one produced."""
+    M, K, H, N = 16, 1024, 2048, 512
+    x = synth.activations(M, K, "normal", 123)
+    w1, w2 = synth.weights(H, K, 124), synth.weights(N, H, 125)
+    ap, sa = oracle.quantize_pack(x, 128)
+    w1p, w1s = oracle.quantize_pack(w1, 128)
+    w2p, w2s = oracle.quantize_pack(w2, 128)
+    hq = torch.empty((M, H // 2), dtype=torch.uint8, device="cuda")
+    hs = torch.empty((M, H // 128), dtype=torch.float16, device="cuda")
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    apex.apex_w4a4_gemm_quant(M, H, K, 128, 128, dev(ap), dev(sa), dev(w1p), dev(w1s), None,
+                              hq, hs, False, apex.workspace(M, H, K))
+    apex.apex_w4a4_gemm(M, N, H, 128, 128, hq, hs, dev(w2p), dev(w2s), y, apex.workspace(M, N, H))
+    torch.cuda.synchronize()
+    check_status(apex)
+    ref = oracle.gemm(host(hq), host(hs), w2p, w2s, M, N, H, 128, 128)
+    assert_close(host(y).astype(np.float64), ref)
