@@ -685,11 +685,10 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
 #pragma unroll
       for (int e = 0; e < C::CPT; ++e) {
         const float v = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
-        float am = fabsf(__half2float(__float2half_rn(v)));
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1)
-          am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
-        if (lane == 0) qmax[w4 * C::CPT + e] = am;
+        // non-negative floats order like their bit patterns: one warp reduction instruction
+        const uint32_t am = __reduce_max_sync(
+            0xffffffffu, __float_as_uint(fabsf(__half2float(__float2half_rn(v)))));
+        if (lane == 0) qmax[w4 * C::CPT + e] = __uint_as_float(am);
       }
       named_bar_sync(FB, NF);
       const int kk = n0t + 32 * w4 + lane;   // this row's K index in the next layer
