@@ -540,7 +540,70 @@ def run_sweep(args, rank, world, local):
             "gemm_TOPS": round(g.ops / (gm * 1e-3) / 1e12, 2),
             "gemm_GBs": round(g.gemm_bytes(activation_form(g.M)) / (gm * 1e-3) / 1e9, 1),
             "roofline": roofline_obj(g, gm, peaks, peaks_kind)})
+    for m in (2048, 16):
+        line = chain_line(apex, torch, m, steps, args.warmup, world)
+        lines.append(line)
     return lines if rank == 0 else None
+
+
+def chain_line(apex, torch, M, steps, warmup, world):
+    """Two chained W4A4 layers (the MLP pair's shapes: 8192 -> 28672 -> 8192), timed as one
+    step two ways: with the first layer's output quantized in its epilogue for the second
+    (apex_w4a4_gemm_quant), and unfused (fp16 output, then the activation quantizer)."""
+    up, down = synth.workloads()["mlp_up_m2048_n28672_k8192"], \
+        synth.workloads()["mlp_down_m2048_n8192_k28672"]
+    K, H, N = up.K, up.N, down.N
+    exp = activation_form(M) == "expanded"
+    dev = torch.device("cuda")
+    x = torch.from_numpy(synth.activations(M, K, "student_t", 7)).to(dev)
+    w1 = torch.from_numpy(synth.weights(H, K, 8)).to(dev)
+    w1p, w1s = apex.pack_weights(w1, 128)
+    del w1
+    w2 = torch.from_numpy(synth.weights(N, H, 9)).to(dev)
+    w2p, w2s = apex.pack_weights(w2, 128)
+    del w2
+    xa = torch.empty((M, K if exp else K // 2), dtype=torch.uint8, device=dev)
+    xs = torch.empty((M, K // 128), dtype=torch.float16, device=dev)
+    ha = torch.empty((M, H if exp else H // 2), dtype=torch.uint8, device=dev)
+    hs = torch.empty((M, H // 128), dtype=torch.float16, device=dev)
+    hy = torch.empty((M, H), dtype=torch.float16, device=dev)
+    y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    ws1, ws2 = apex.workspace(M, H, K), apex.workspace(M, N, H)
+    quant = apex.apex_quantize_act_int4_expanded if exp else apex.apex_quantize_act_int4
+    gemm = apex.apex_w4a4_gemm_expanded if exp else apex.apex_w4a4_gemm
+    gemm_q = apex.apex_w4a4_gemm_expanded_quant if exp else apex.apex_w4a4_gemm_quant
+
+    def fused(i, s):
+        quant(x, M, K, 128, xa, xs, s)
+        gemm_q(M, H, K, 128, 128, xa, xs, w1p, w1s, None, ha, hs, exp, ws1, None, s)
+        gemm(M, N, H, 128, 128, ha, hs, w2p, w2s, y, ws2, None, s)
+
+    def unfused(i, s):
+        quant(x, M, K, 128, xa, xs, s)
+        gemm(M, H, K, 128, 128, xa, xs, w1p, w1s, hy, ws1, None, s)
+        quant(hy, M, H, 128, ha, hs, s)
+        gemm(M, N, H, 128, 128, ha, hs, w2p, w2s, y, ws2, None, s)
+
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        fused(i, stream)
+        unfused(i, stream)
+    torch.cuda.synchronize()
+    if apex.apex_get_device_status() != 0:
+        raise RuntimeError("device status not clean after the chain warm-up")
+    f_ms, _ = timed_graph(torch, fused, steps, warmup, world)
+    u_ms, _ = timed_graph(torch, unfused, steps, warmup, world)
+    f_ms = max_over_ranks(f_ms / steps, world)
+    u_ms = max_over_ranks(u_ms / steps, world)
+    ops = 2.0 * M * K * H + 2.0 * M * H * N
+    return {"sweep": f"mlp_chain_m{M}", "M": M, "K": K, "hidden": H, "N": N,
+            "activation_form": activation_form(M), "steps": steps,
+            "fused_step_ms": round(f_ms, 5), "unfused_step_ms": round(u_ms, 5),
+            "fused_TOPS": round(job_throughput(ops, f_ms, world), 2),
+            "unfused_TOPS": round(job_throughput(ops, u_ms, world), 2),
+            "what": ("x -> quantize -> up (8192 -> 28672) -> down (28672 -> 8192); fused: the "
+                     "up layer writes the down layer's int4 operand in its epilogue; unfused: "
+                     "fp16 output, then the activation quantizer")}
 
 
 def p_copies(g, l2):
