@@ -216,7 +216,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, si
 
 template <int BT, int MODE, bool QOUT>
 apex_status_t launch_bt(const Plan& p, const Maps& m, GemmArgs a, cudaStream_t s) {
-  using C = GemmCfg<BT, MODE>;
+  using C = GemmCfg<BT, MODE, QOUT>;
   auto kern = apex::w4a4_gemm_kernel<BT, MODE, QOUT>;
   static thread_local int attr_dev = -1;   // the attribute is per device; set it once each
   int dev = 0;
@@ -388,7 +388,7 @@ apex_status_t gemm_entry(bool a_expanded, int64_t M, int64_t N, int64_t K, int32
   if (qo.q && N % 128) return APEX_ERR_UNSUPPORTED;   // the output's groups are whole tiles
   if (!aligned(a_q, 16) || !aligned(w_packed, 16) || !aligned(a_scales, 2) ||
       !aligned(w_scales, 2) || (y_f16 && !aligned(y_f16, 2)) ||
-      (qo.q && (!aligned(qo.q, 4) || !aligned(qo.scales, 2))) ||
+      (qo.q && (!aligned(qo.q, 16) || !aligned(qo.scales, 2))) ||
       (workspace && !aligned(workspace, 256)))
     return APEX_ERR_ALIGNMENT;
 

@@ -128,7 +128,7 @@ __host__ __device__ constexpr int stage_groups(int bt) { return bt <= 32 ? 4 : 2
 // in shared memory: the narrow tiles of decode-sized batches.
 __host__ __device__ constexpr int max_cluster(int bt) { return bt == 16 ? 4 : bt == 32 ? 2 : 1; }
 
-template <int BT, int MODE>
+template <int BT, int MODE, bool QOUT = false>
 struct GemmCfg {
   static constexpr bool AQ8 = MODE == MODE_AQ8;
   static constexpr int BM = 128;
@@ -172,7 +172,13 @@ struct GemmCfg {
   static constexpr int OFF_SAT = OFF_XA + NX * XA;
   static constexpr int OFF_RED = OFF_SAT + SAT;
   static constexpr int OFF_RCV = OFF_RED + RED;
-  static constexpr int OFF_BAR = OFF_RCV + RCV;
+  // the quantized output's fp16 tile [BT tokens][BM rows] on its way from row-per-thread to
+  // token-per-thread: narrow tiles stage it in the second team's sum buffer (idle by then),
+  // wide tiles get a buffer of their own (left out of the stage budget above)
+  static constexpr int STG = QOUT && TEAMS == 1 ? BT * BM * 2 : 0;
+  static_assert(!QOUT || TEAMS == 1 || RED >= BT * BM * 2, "staging in the sum buffer");
+  static constexpr int OFF_STG = OFF_RCV + RCV;
+  static constexpr int OFF_BAR = OFF_STG + STG;
   // Hand-off unit: the groups that pass between converters, MMA and epilogue under one
   // barrier phase -- a whole stage for narrow tiles (the MMA issue loop is short on work
   // per group there), a single group for wide ones (whose partial slots fill TMEM).
@@ -289,10 +295,10 @@ __device__ __forceinline__ bool get_seg(const GemmArgs& a, int k, Seg& sg) {
 // QOUT: the quantized output (args.qout) is written; a separate instantiation, so plain
 // GEMMs carry none of its code.
 template <int BT, int MODE, bool QOUT = false>
-__global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
+__global__ void __launch_bounds__(GemmCfg<BT, MODE, QOUT>::THREADS, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmW,
                      const __grid_constant__ CUtensorMap tmA, const GemmArgs args) {
-  using C = GemmCfg<BT, MODE>;
+  using C = GemmCfg<BT, MODE, QOUT>;
   constexpr bool DUMP = MODE == MODE_DUMP;
   constexpr bool AQ8 = C::AQ8;
   extern __shared__ uint8_t smem_raw[];
@@ -313,6 +319,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
   uint64_t* mma_done = d_empty + C::NDU;
   uint64_t* rcv_full = mma_done + 1;   // a cluster owner: every partner's part has landed
   float* s_rcv = reinterpret_cast<float*>(smem + C::OFF_RCV);
+  uint8_t* s_stg = C::TEAMS == 2 ? reinterpret_cast<uint8_t*>(s_red) : smem + C::OFF_STG;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* s_abort = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
   int* s_last = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
@@ -677,53 +684,73 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE>::THREADS, 1)
         }
       }
       if constexpr (!QOUT) return;
-      // each token's absmax over the tile's 128 rows: a warp's 32 rows by shuffles, then
-      // the four warps of this column block through shared memory (the first token-scale
-      // buffer of this team, idle between segments)
-      float* qmax = s_sat + h * 4 * C::CPT;   // [lane quarter][CPT]
-      const int w4 = warp & 3;
+      // The quantized output is made token by token.  The tile goes through shared memory
+      // as fp16 [token][128 rows]; then TPT neighbouring threads take one token's 128
+      // values, RPT each, find the group's absmax with a few shuffles and quantize with the
+      // activation quantizer's own routines: one scale per token, independent divisions,
+      // whole words stored.  The 16-byte chunks of a token's line are permuted (chunk c
+      // lives at c ^ ((token * TPT + c / R8) & 7)) so that the row-per-thread writes and the
+      // token-per-thread 16-byte reads both meet every bank once per phase.
+      constexpr int TPT = NF / BT;               // threads per token
+      constexpr int RPT = C::BM / TPT;           // values (the next layer's k) per thread
+      constexpr int R8 = RPT / 8;                // their 16-byte chunks
+      static_assert(NF % BT == 0 && 32 % TPT == 0 && R8 >= 2, "token-per-thread mapping");
+      auto chunk_at = [&](int tok, int c) {
+        return tok * (C::BM * 2) + ((c ^ ((tok * TPT + c / R8) & 7)) << 4);
+      };
+      // narrow tiles stage in the sum buffer: every thread has read its sums out of it
+      if constexpr (C::TEAMS == 2) named_bar_sync(FB, NF);
 #pragma unroll
       for (int e = 0; e < C::CPT; ++e) {
         const float v = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
-        // non-negative floats order like their bit patterns: one warp reduction instruction
-        const uint32_t am = __reduce_max_sync(
-            0xffffffffu, __float_as_uint(fabsf(__half2float(__float2half_rn(v)))));
-        if (lane == 0) qmax[w4 * C::CPT + e] = __uint_as_float(am);
+        *reinterpret_cast<__half*>(s_stg + chunk_at(h * C::CPT + e, row >> 3) +
+                                   2 * (row & 7)) = __float2half_rn(v);
       }
       named_bar_sync(FB, NF);
-      const int kk = n0t + 32 * w4 + lane;   // this row's K index in the next layer
+      {
+        const int tok = et / TPT, part = et % TPT;
+        uint4 v[R8];
 #pragma unroll
-      for (int e = 0; e < C::CPT; ++e) {
-        const int m = m0t + h * C::CPT + e;
-        const float am = fmaxf(fmaxf(qmax[e], qmax[C::CPT + e]),
-                               fmaxf(qmax[2 * C::CPT + e], qmax[3 * C::CPT + e]));
-        const __half sc = group_scale(am);
-        const float v = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
-        const int qv = quant1(__half2float(__float2half_rn(v)), __half2float(sc));
-        // one byte per lane (packed: the even lanes hold k and k+1), then four bytes per word
-        uint32_t b;
-        if (args.qexp) {
-          b = ((uint32_t)qv & 15u) << 4;
-        } else {
-          const int qn = __shfl_down_sync(0xffffffffu, qv, 1);
-          b = ((uint32_t)qv & 15u) | (((uint32_t)qn & 15u) << 4);
+        for (int j = 0; j < R8; ++j)
+          v[j] = *reinterpret_cast<const uint4*>(s_stg + chunk_at(tok, part * R8 + j));
+        __half2 mx = __float2half2_rn(0.0f);
+#pragma unroll
+        for (int j = 0; j < R8; ++j) {
+          const __half2* hv = reinterpret_cast<const __half2*>(&v[j]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) mx = __hmax2(mx, __habs2(hv[i]));
         }
-        const uint32_t wd = b | (__shfl_down_sync(0xffffffffu, b, 2) << 8) |
-                            (__shfl_down_sync(0xffffffffu, b, 4) << 16) |
-                            (__shfl_down_sync(0xffffffffu, b, 6) << 24);
+        float am = fmaxf(__low2float(mx), __high2float(mx));
+#pragma unroll
+        for (int o = 1; o < TPT; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+        const __half sc = group_scale(am);
+        const float sf = __half2float(sc);
+        const int m = m0t + tok;
         if (m < M) {
           if (args.qexp) {
-            // lane 8c: k = 8c, 8c+2, 8c+4, 8c+6 of the chunk; lane 8c+1: the odd k
-            if ((lane & 7) < 2)
-              *reinterpret_cast<uint32_t*>(args.qout + (size_t)m * N + (kk & ~7) +
-                                           4 * (lane & 1)) = wd;
-          } else if ((lane & 7) == 0) {
-            *reinterpret_cast<uint32_t*>(args.qout + (size_t)m * (N / 2) + kk / 2) = wd;
+            uint8_t* dst = args.qout + (size_t)m * N + n0t + part * RPT;
+#pragma unroll
+            for (int j = 0; j < R8; j += 2) {
+              const uint2 x0 = quant_expand8(v[j], sf), x1 = quant_expand8(v[j + 1], sf);
+              *reinterpret_cast<uint4*>(dst + 8 * j) = make_uint4(x0.x, x0.y, x1.x, x1.y);
+            }
+          } else {
+            uint8_t* dst = args.qout + (size_t)m * (N / 2) + n0t / 2 + part * (RPT / 2);
+            if constexpr (R8 == 2) {
+              *reinterpret_cast<uint2*>(dst) =
+                  make_uint2(quant_pack8(v[0], sf), quant_pack8(v[1], sf));
+            } else {
+#pragma unroll
+              for (int j = 0; j < R8; j += 4)
+                *reinterpret_cast<uint4*>(dst + 4 * j) =
+                    make_uint4(quant_pack8(v[j], sf), quant_pack8(v[j + 1], sf),
+                               quant_pack8(v[j + 2], sf), quant_pack8(v[j + 3], sf));
+            }
           }
-          if (w4 == 0 && lane == 0) args.qscale[(size_t)m * (N / 128) + n0t / 128] = sc;
+          if (part == 0) args.qscale[(size_t)m * (N / 128) + n0t / 128] = sc;
         }
       }
-      named_bar_sync(FB, NF);   // qmax is free again
+      named_bar_sync(FB, NF);   // the staging buffer is free again
     };
     // Narrow tiles pipeline the partial loads within a hand-off unit.
     constexpr bool PIPE = C::CPT == 16 && C::GPB > 1;

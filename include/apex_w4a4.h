@@ -114,7 +114,8 @@ apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, i
  * the fp16 Y this call computes -- every tile of 128 outputs is one K-group of the next
  * layer, so its scale and codes are made in the GEMM's epilogue.
  *   y_f16 may be NULL (then only yq and yq_scales are written).  Requires N % 128 == 0
- *   (APEX_ERR_UNSUPPORTED otherwise); yq 4-byte and yq_scales 2-byte aligned.
+ *   (APEX_ERR_UNSUPPORTED otherwise); yq 16-byte (as the next GEMM's operand needs) and
+ *   yq_scales 2-byte aligned.
  */
 apex_status_t apex_w4a4_gemm_quant(int64_t M, int64_t N, int64_t K, int32_t group_a,
                                    int32_t group_w, const void *a_packed, const void *a_scales,

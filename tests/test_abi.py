@@ -83,6 +83,18 @@ def test_quantizer_argument_errors_are_host_side(lib):
     assert pw(P(0x1000), 4, 256, 128, P(0x2002), P(0x3000), None) == apex.APEX_ERR_ALIGNMENT
 
 
+def test_quantized_output_argument_errors_are_host_side(lib):
+    def f(N=256, y=None, yq=0x6000, yqs=0x7000):
+        return lib.apex_w4a4_gemm_quant(16, N, 256, 128, 128, P(0x1000), P(0x2000), P(0x3000),
+                                        P(0x4000), P(y), P(yq), P(yqs), 0, None, 0, None)
+    assert f(N=200) == apex.APEX_ERR_UNSUPPORTED          # output groups are whole tiles
+    assert f(yq=None) == apex.APEX_ERR_INVALID_ARG
+    assert f(yqs=None) == apex.APEX_ERR_INVALID_ARG
+    assert f(yq=0x6008) == apex.APEX_ERR_ALIGNMENT        # written in 16-byte words
+    assert f(yqs=0x7001) == apex.APEX_ERR_ALIGNMENT
+    assert f(y=0x5001) == apex.APEX_ERR_ALIGNMENT
+
+
 def test_partials_argument_errors(lib):
     f = lib.apex_w4a4_group_partials
     assert f(4, 8, 100, P(0x1000), P(0x2000), P(0x3000), None) == apex.APEX_ERR_INVALID_ARG
