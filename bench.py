@@ -628,7 +628,10 @@ def run_reference(args, rank, world):
     cb["value"] = v
     return {"metric": "W4A4-g128 GEMM effective TOPS (quantize + GEMM step) and % of roofline",
             "value": v, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup,
+            # one whole step of the workload at the sampled rate
+            "ms_per_step": round(g.ops / (v * 1e12) * 1e3, 3) if v > 0 else None,
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int64 partials, fp64 scaling", "data": "synthetic",
             "config": {"workload": g.name, "M": g.M, "N": g.N, "K": g.K, "group_a": 128,
                        "group_w": g.gw},
