@@ -479,6 +479,8 @@ QUANT_OUT_SHAPES = [
     (64, 1024, 512),
     (100, 512, 768),
     (200, 384, 1024),    # 128-token tiles, ragged token block
+    (16, 12800, 1024),   # stream-K: 200 units over 148 CTAs, pieces of two tiles per CTA
+    (200, 6400, 1024),   # stream-K with 128-token tiles
 ]
 
 
@@ -556,3 +558,42 @@ def test_chained_layers_through_the_quantized_output(apex):
     check_status(apex)
     ref = oracle.gemm(host(hq), host(hs), w2p, w2s, M, N, H, 128, 128)
     assert_close(host(y).astype(np.float64), ref)
+
+
+@pytest.mark.parametrize("M", [2048, 16])
+def test_gemm_quantized_output_full_size_sampled_rows(apex, M):
+    """The up-projection of the MLP pair (8192 -> 28672) at full size, in the form the chained
+    step times (expanded activations from M = 128 on): sampled rows of Y meet the GEMM bar,
+    and the same rows of the quantized output, in both output forms, are the oracle's
+    quantizer applied to Y, bit for bit."""
+    K, N = 8192, 28672
+    x = synth.activations(M, K, "student_t", 7)
+    w = synth.weights(N, K, 8)
+    wp, sw = apex.pack_weights(dev(w), 128)
+    expanded_in = M >= 128
+    if expanded_in:
+        a_q, a_s = apex.quantize_act_expanded(dev(x), 128)
+        fn = apex.apex_w4a4_gemm_expanded_quant
+    else:
+        a_q, a_s = apex.quantize_act(dev(x), 128)
+        fn = apex.apex_w4a4_gemm_quant
+    ws = apex.workspace(M, N, K)
+    rows = np.array(sorted({r for r in (0, 1, 127, 128, M // 3, M - 1) if r < M}), dtype=np.int64)
+    ap_ref, sa_ref = oracle.quantize_pack(x[rows], 128)
+    ref = oracle.gemm(ap_ref, sa_ref, host(wp), host(sw), rows.size, N, K, 128, 128)
+    for expanded_out in (False, True):
+        y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+        yq = torch.empty((M, N if expanded_out else N // 2), dtype=torch.uint8, device="cuda")
+        ys = torch.empty((M, N // 128), dtype=torch.float16, device="cuda")
+        fn(M, N, K, 128, 128, a_q, a_s, wp, sw, y, yq, ys, expanded_out, ws)
+        torch.cuda.synchronize()
+        check_status(apex)
+        y_rows = host(y)[rows]
+        assert_close(y_rows.astype(np.float64), ref)
+        q_ref, s_ref = oracle.quantize_pack(y_rows, 128)
+        if expanded_out:
+            want = expected_expanded(oracle.unpack(q_ref, N).astype(np.int64))
+        else:
+            want = q_ref
+        assert np.array_equal(host(yq)[rows], want)
+        assert np.array_equal(f16(ys)[rows], s_ref.view(np.uint16))
