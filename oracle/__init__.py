@@ -16,6 +16,10 @@ Parity status per function (pins in ``tests/test_oracle_pins.py``):
   group_partials    pinned (numpy int64 matmul per group)
   gemm              pinned (fp64 brute force of dequantised operands, group=K closed
                     form, permutation invariance, power-of-two linearity)
+  split_outlier_channels, gemm_dual
+                    pinned (outlier-only inputs reduce to numpy's fp64 matmul; no
+                    outlier channels reduce to gemm; the per-element error bound of the
+                    dual path against the exact product; planted mistakes fail it)
 """
 from __future__ import annotations
 
@@ -173,6 +177,43 @@ def gemm(ap, sa, wp, sw, M, N, K, ga, gw, rows=None) -> np.ndarray:
     if rc:
         raise ValueError(f"oracle gemm failed (rc={rc})")
     return y
+
+
+def split_outlier_channels(x: np.ndarray, channels):
+    """The activation split of the outlier dual path ("OSC: Hardware Efficient W4A4
+    Quantization via Outlier Separation in Channel Dimension", abstract): a fixed set of
+    input channels, the same for every token, is pulled out into a compact dense fp16
+    tensor for the 16-bit branch, and the 4-bit path sees those channels as zeros.
+
+    x: [rows, K] float16; channels: distinct indices in [0, K).
+    Returns (x_in float16 [rows, K] with the channels zeroed, x_out float16
+    [rows, len(channels)] holding them in the given order)."""
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.float16 or x.ndim != 2:
+        raise TypeError("x must be a 2-D float16 array")
+    ch = np.asarray(channels, dtype=np.int64)
+    if ch.size and (ch.min() < 0 or ch.max() >= x.shape[1] or np.unique(ch).size != ch.size):
+        raise ValueError("channels must be distinct indices of x's columns")
+    x_in = x.copy()
+    x_in[:, ch] = 0
+    return x_in, np.ascontiguousarray(x[:, ch])
+
+
+def gemm_dual(ap, sa, wp, sw, x_out, w_out, M, N, K, ga, gw, rows=None) -> np.ndarray:
+    """The dual-path output (OSC abstract): the W4A4 path on the quantized operands,
+    Y4 = gemm(ap, sa, wp, sw, ...), plus the 16-bit branch over the outlier channels,
+    x_out [M, C] . w_out [N, C]^T, the fp16 values multiplied exactly and summed in fp64
+    (numpy matmul as the library step).  [len(rows) or M, N] float64."""
+    y = gemm(ap, sa, wp, sw, M, N, K, ga, gw, rows)
+    xo = np.asarray(x_out)
+    wo = np.asarray(w_out)
+    if xo.dtype != np.float16 or wo.dtype != np.float16:
+        raise TypeError("the 16-bit branch operands must be float16")
+    if xo.shape[0] != M or wo.shape[0] != N or xo.shape[1] != wo.shape[1]:
+        raise ValueError("x_out must be [M, C] and w_out [N, C]")
+    if rows is not None:
+        xo = xo[np.asarray(rows, dtype=np.int64)]
+    return y + xo.astype(np.float64) @ wo.astype(np.float64).T
 
 
 def within_tolerance(y, y_ref, max_abs_ref=None):

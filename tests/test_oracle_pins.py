@@ -324,6 +324,129 @@ def test_brute_force_pin_catches_planted_mistakes(oracle_mod):
     assert bad3.shape == ref.shape and np.max(np.abs(bad3 - ref)) > tol
 
 
+# ------------------------------------------------------------------ outlier dual path
+# "OSC: Hardware Efficient W4A4 Quantization via Outlier Separation in Channel Dimension",
+# abstract: fixed outlier channels go through a 16-bit branch GEMM, the rest through the
+# 4-bit GEMM.
+
+
+def _dual_inputs(rng, M, N, K, n_out, boost=20.0):
+    ch = np.sort(rng.choice(K, size=n_out, replace=False))
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[:, ch] *= np.float32(boost)
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    return x.astype(np.float16), w.astype(np.float16), ch
+
+
+def _dual_by_oracle(oracle_mod, x, w, ch, gw=128):
+    M, K = x.shape
+    N = w.shape[0]
+    x_in, x_out = oracle_mod.split_outlier_channels(x, ch)
+    ap, sa = oracle_mod.quantize_pack(x_in, 128)
+    wp, sw = oracle_mod.quantize_pack(w, gw)
+    y = oracle_mod.gemm_dual(ap, sa, wp, sw, x_out, np.ascontiguousarray(w[:, ch]),
+                             M, N, K, 128, gw)
+    return y, (ap, sa, wp, sw)
+
+
+def _mixed_reference(x, w, ch, ops, gw=128):
+    """Element-level restatement on full-width operands: channel k contributes
+    x[m,k] w[n,k] (fp16 values) when it is an outlier channel, else the product of the
+    dequantised int4 values; one fp64 matmul of the two mixed matrices."""
+    ap, sa, wp, sw = ops
+    K = x.shape[1]
+    xd = dequant(np_unpack(ap, K), sa, 128)
+    wd = dequant(np_unpack(wp, K), sw, gw)
+    mask = np.zeros(K, dtype=bool)
+    mask[ch] = True
+    xm = np.where(mask[None, :], x.astype(np.float64), xd)
+    wm = np.where(mask[None, :], w.astype(np.float64), wd)
+    return xm @ wm.T
+
+
+@pytest.mark.parametrize("gw", [128, 512])
+def test_dual_path_matches_element_level_restatement(oracle_mod, gw):
+    rng = np.random.default_rng(61)
+    x, w, ch = _dual_inputs(rng, 7, 9, 1024, 11)
+    y, ops = _dual_by_oracle(oracle_mod, x, w, ch, gw)
+    ref = _mixed_reference(x, w, ch, ops, gw)
+    assert np.max(np.abs(y - ref)) <= 1e-12 * np.max(np.abs(ref))
+    # the 4-bit operands see the outlier channels as zeros
+    assert not np.any(np_unpack(ops[0], 1024)[:, ch])
+
+
+def test_dual_path_outlier_only_input_is_the_fp16_product(oracle_mod):
+    rng = np.random.default_rng(62)
+    x, w, ch = _dual_inputs(rng, 5, 6, 512, 9)
+    only = np.zeros_like(x)
+    only[:, ch] = x[:, ch]
+    y, ops = _dual_by_oracle(oracle_mod, only, w, ch)
+    assert not np.any(ops[1].astype(np.float32))       # every group scale is 0
+    ref = only.astype(np.float64) @ w.astype(np.float64).T
+    assert np.max(np.abs(y - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_dual_path_without_outlier_channels_is_the_w4a4_gemm(oracle_mod):
+    rng = np.random.default_rng(63)
+    x, w, _ = _dual_inputs(rng, 4, 5, 384, 3)
+    y, ops = _dual_by_oracle(oracle_mod, x, w, np.array([], dtype=np.int64))
+    ap, sa, wp, sw = ops
+    assert np.array_equal(y, oracle_mod.gemm(ap, sa, wp, sw, 4, 5, 384, 128, 128))
+
+
+def test_dual_path_cuts_the_error_of_outlier_channels(oracle_mod):
+    """What the dual path is for: on token-persistent outlier channels the error against
+    the exact product of the fp16 operands drops well below the single 4-bit path's."""
+    M, N, K = 8, 16, 2048
+    x = synth.activations(M, K, "outlier", 5)
+    w = synth.weights(N, K, 5)
+    ch = synth.outlier_channels(K, 5 * 16 + 2)
+    exact = x.astype(np.float64) @ w.astype(np.float64).T
+    dual, _ = _dual_by_oracle(oracle_mod, x, w, ch)
+    ap, sa = oracle_mod.quantize_pack(x, 128)
+    wp, sw = oracle_mod.quantize_pack(w, 128)
+    single = oracle_mod.gemm(ap, sa, wp, sw, M, N, K, 128, 128)
+    e_dual = np.sqrt(np.mean((dual - exact) ** 2))
+    e_single = np.sqrt(np.mean((single - exact) ** 2))
+    assert e_dual < 0.5 * e_single
+
+
+def test_dual_pin_catches_planted_mistakes(oracle_mod):
+    """Plausible mistakes in the dual path, planted on the CPU, each fail the
+    element-level restatement: outliers left in the 4-bit operands, the 16-bit branch
+    dropped, and branch weights taken in the wrong channel order."""
+    rng = np.random.default_rng(64)
+    M, N, K = 6, 8, 1024
+    x, w, ch = _dual_inputs(rng, M, N, K, 11)
+    y, ops = _dual_by_oracle(oracle_mod, x, w, ch)
+    ref = _mixed_reference(x, w, ch, ops)
+    tol = 1e-12 * np.max(np.abs(ref))
+    assert np.max(np.abs(y - ref)) <= tol
+    ap, sa, wp, sw = ops
+    x_out = np.ascontiguousarray(x[:, ch])
+    w_out = np.ascontiguousarray(w[:, ch])
+    # outliers not zeroed before quantizing (counted on both paths)
+    ap_bad, sa_bad = oracle_mod.quantize_pack(x, 128)
+    bad = oracle_mod.gemm_dual(ap_bad, sa_bad, wp, sw, x_out, w_out, M, N, K, 128, 128)
+    assert np.max(np.abs(bad - ref)) > tol
+    # the branch dropped
+    assert np.max(np.abs(oracle_mod.gemm(ap, sa, wp, sw, M, N, K, 128, 128) - ref)) > tol
+    # branch weights in reverse channel order
+    bad = oracle_mod.gemm_dual(ap, sa, wp, sw, x_out, np.ascontiguousarray(w_out[:, ::-1]),
+                               M, N, K, 128, 128)
+    assert np.max(np.abs(bad - ref)) > tol
+
+
+def test_split_outlier_channels_argument_rules(oracle_mod):
+    x = np.zeros((2, 8), dtype=np.float16)
+    with pytest.raises(ValueError):
+        oracle_mod.split_outlier_channels(x, [1, 1])
+    with pytest.raises(ValueError):
+        oracle_mod.split_outlier_channels(x, [8])
+    with pytest.raises(TypeError):
+        oracle_mod.split_outlier_channels(x.astype(np.float32), [1])
+
+
 def test_tolerance_rule():
     ok, _ = __import__("oracle").within_tolerance([1.0, 2.0], [1.0, 2.001])
     assert ok
