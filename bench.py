@@ -34,6 +34,10 @@ from group_quantized_w4a4_b200 import roofline, synth  # noqa: E402
 DEFAULT_WORKLOAD = "decode_m16_n8192_k8192"
 SECOND_WORKLOAD = "prefill_m4096_n8192_k8192"
 INT8_PER_BF16 = 2.0   # nominal dense int8 : bf16 tensor throughput ratio on B200 (4.5 : 2.25)
+INT8_SPEC_TOPS = 4500.0   # B200 dense int8 tensor throughput, public spec (context)
+HBM_SPEC_GBS = 8000.0     # B200 HBM3e, public spec (context)
+PREROLL_S = 0.1           # untimed replays under the clock sampler before a timed replay
+PREFILL_STEPS = 100       # the tensor-bound companion line's timed steps (about 70 ms)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -99,6 +103,8 @@ class ClockSampler:
     def __init__(self, cuda_index: int):
         self.cuda_index = cuda_index
         self.samples = []
+        self.stamps = []
+        self.timed = None       # (t0, t1) host clock around the timed replay
         self.reasons = 0
         self.max_mhz = None
         self._stop = None
@@ -135,6 +141,7 @@ class ClockSampler:
             while not self._stop.is_set():
                 try:
                     self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    self.stamps.append(time.perf_counter())
                     self.reasons |= int(get_reasons(h))
                 except Exception:
                     pass
@@ -150,9 +157,16 @@ class ClockSampler:
         self._stop.set()
         self._thread.join(timeout=2)
         names = sorted(v for k, v in self.REASONS.items() if self.reasons & k)
+        in_timed = 0
+        if self.timed is not None:
+            t0, t1 = self.timed
+            in_timed = sum(1 for t in self.stamps if t0 <= t <= t1)
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
-                "sm_max_mhz": self.max_mhz, "samples": len(self.samples), "reasons": names,
-                "source": "NVML polled every 2 ms during the timed region"}
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "samples_in_timed_replay": in_timed, "reasons": names,
+                "source": ("NVML polled every 2 ms while the GPU ran the same CUDA graph: "
+                           f"{PREROLL_S * 1e3:.0f} ms of untimed replays right before the timed "
+                           "replay, then the timed replay itself")}
 
 
 # ------------------------------------------------------------------ the apex arm
@@ -238,17 +252,31 @@ def timed_graph(torch, fn, steps, first, world, clocks=None):
         graph.replay()
     torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if clocks:
+        # the clock record covers the GPU under this same load: untimed replays for
+        # PREROLL_S first (a short timed region alone leaves NVML too few samples)
+        clocks.start()
+        t_end = time.perf_counter() + PREROLL_S
+        with torch.cuda.stream(side):
+            while time.perf_counter() < t_end:
+                graph.replay()
+                side.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    if clocks:
-        clocks.start()
+    t0 = time.perf_counter()
     with torch.cuda.stream(side):
         start.record(side)
         graph.replay()
         stop.record(side)
     torch.cuda.synchronize()
+    t1 = time.perf_counter()
     barrier(world)
-    clk = clocks.stop() if clocks else None
+    clk = None
+    if clocks:
+        clocks.timed = (t0, t1)
+        clk = clocks.stop()
+        if clk.get("sm_mhz"):
+            clk["ms_x_sm_mhz"] = round(start.elapsed_time(stop) * clk["sm_mhz"], 3)
     del graph
     return start.elapsed_time(stop), clk
 
@@ -371,10 +399,40 @@ def recorded_traffic(name: str):
     return rec.get("traffic_bytes_per_launch", {}).get(name)
 
 
-def roofline_obj(g, gemm_ms_avg, peaks, peaks_kind, traffic=None):
+def measure_int8_peak(torch, reps: int = 10):
+    """Dense int8 tensor throughput of this GPU, measured: torch._int_mm (cuBLASLt) on
+    8192^3 int8 operands, best of `reps` launches timed with CUDA events (TOPS)."""
+    n = 8192
+    a = torch.randint(-8, 8, (n, n), dtype=torch.int8, device="cuda")
+    b = torch.randint(-8, 8, (n, n), dtype=torch.int8, device="cuda")
+    for _ in range(3):
+        torch._int_mm(a, b.t())
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(reps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        torch._int_mm(a, b.t())
+        e.record()
+        torch.cuda.synchronize()
+        best = min(best, s.elapsed_time(e))
+    del a, b
+    torch.cuda.empty_cache()
+    return {"tops": round(2.0 * n ** 3 / (best * 1e-3) / 1e12, 1),
+            "how": f"torch._int_mm int8 {n}^3, best of {reps}, CUDA events, in this run"}
+
+
+def roofline_obj(g, gemm_ms_avg, peaks, peaks_kind, traffic=None, int8_peak=None,
+                 form=None):
     hbm = float(peaks["hbm_gbs"]) * 1e9
-    i8 = float(peaks.get("bf16_tflops", 1590.0)) * 1e12 * INT8_PER_BF16
-    nbytes = g.gemm_bytes(activation_form(g.M))
+    if int8_peak is not None:
+        i8 = float(int8_peak["tops"]) * 1e12
+        i8_note = f"int8 measured: {int8_peak['how']}"
+    else:
+        i8 = float(peaks.get("bf16_tflops", 1590.0)) * 1e12 * INT8_PER_BF16
+        i8_note = (f"int8 = {INT8_PER_BF16:g} x bf16_tflops of {peaks_kind} "
+                   "(nominal int8:bf16 ratio)")
+    nbytes = g.gemm_bytes(form or activation_form(g.M))
     t_bound, bound = roofline.bound_time_s(g.ops, nbytes, i8, hbm)
     t = gemm_ms_avg * 1e-3
     if bound == "hbm":
@@ -382,15 +440,17 @@ def roofline_obj(g, gemm_ms_avg, peaks, peaks_kind, traffic=None):
         peak = float(peaks["hbm_gbs"])
         unit = "GB/s"
         note = f"hbm_gbs of {peaks_kind}"
+        spec = {"peak": HBM_SPEC_GBS, "frac": round(achieved / HBM_SPEC_GBS, 4)}
     else:
         achieved = g.ops / t / 1e12
         peak = i8 / 1e12
         unit = "TOPS"
-        note = f"int8 = {INT8_PER_BF16:g} x bf16_tflops of {peaks_kind} (nominal int8:bf16 ratio)"
+        note = i8_note
+        spec = {"peak": INT8_SPEC_TOPS, "frac": round(achieved / INT8_SPEC_TOPS, 4)}
     return {"bound": "hbm" if bound == "hbm" else "tensor", "achieved": round(achieved, 2),
             "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
             "traffic": traffic if traffic is not None else recorded_traffic(g.name),
-            "peak_source": note,
+            "peak_source": note, "spec": spec,
             "algorithmic_bytes": nbytes, "ops": g.ops,
             "kernel_ms": round(gemm_ms_avg, 5)}
 
@@ -451,6 +511,7 @@ def run_apex(args, rank, world, local):
     l2 = int(getattr(props, "L2_cache_size", 126 * 1024 * 1024))
     peaks, peaks_kind = load_peaks()
     g = synth.workloads()[args.workload]
+    int8_peak = measure_int8_peak(torch)
     clocks = ClockSampler(local) if rank == 0 else None
     p, total_ms, gemm_avg, clk, quant_avg = time_workload(apex, torch, g, args.steps,
                                                           args.warmup, world, l2, clocks)
@@ -464,16 +525,18 @@ def run_apex(args, rank, world, local):
     extra = {}
     if not args.no_second and args.workload != SECOND_WORKLOAD:
         g2 = synth.workloads()[SECOND_WORKLOAD]
-        p2, tot2, gm2, _, qm2 = time_workload(apex, torch, g2, max(3, args.steps // 4),
-                                              args.warmup, world, l2)
+        clocks2 = ClockSampler(local) if rank == 0 else None
+        p2, tot2, gm2, clk2, qm2 = time_workload(apex, torch, g2, PREFILL_STEPS,
+                                                 args.warmup, world, l2, clocks2)
         gm2, qm2 = max_over_ranks(gm2, world), max_over_ranks(qm2, world)
-        ms2 = max_over_ranks(tot2 / max(3, args.steps // 4), world)
+        ms2 = max_over_ranks(tot2 / PREFILL_STEPS, world)
         extra[SECOND_WORKLOAD] = {
             "value": round(job_throughput(g2.ops, ms2, world), 2), "unit": "TOPS",
-            "ms_per_step": round(ms2, 4),
+            "ms_per_step": round(ms2, 4), "steps": PREFILL_STEPS,
             "activation_form": activation_form(g2.M),
             "quantize_ms": round(qm2, 5), "gemm_ms": round(gm2, 5),
-            "roofline": roofline_obj(g2, gm2, peaks, peaks_kind)}
+            "roofline": roofline_obj(g2, gm2, peaks, peaks_kind, int8_peak=int8_peak),
+            "clocks": clk2}
         del p2
     if rank != 0:
         return None
@@ -488,7 +551,8 @@ def run_apex(args, rank, world, local):
                    "group_w": g.gw, "parallelism": f"replicas x{world}",
                    "activation_form": form,
                    "l2": f"inputs larger than L2: {p_copies(g, l2)} rotating copies"},
-        "roofline": roofline_obj(g, gemm_avg, peaks, peaks_kind),
+        "roofline": roofline_obj(g, gemm_avg, peaks, peaks_kind, int8_peak=int8_peak),
+        "int8_peak_measured": int8_peak,
         "e2e": {"value": round(job_throughput(g.ops, e2e_ms, world), 3), "unit": "TOPS",
                 "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db,
                 "ms_per_step": round(e2e_ms, 4),
@@ -524,6 +588,7 @@ def run_sweep(args, rank, world, local):
     peaks, peaks_kind = load_peaks()
     names = [n for n in synth.workloads() if n.startswith("sweep_") or n.startswith("mlp_")]
     steps = max(3, args.steps // 4)
+    int8_peak = measure_int8_peak(torch)
     lines = []
     for name in names:
         g = synth.workloads()[name]
@@ -539,7 +604,7 @@ def run_sweep(args, rank, world, local):
             "step_TOPS": round(job_throughput(g.ops, ms, world), 2),
             "gemm_TOPS": round(g.ops / (gm * 1e-3) / 1e12, 2),
             "gemm_GBs": round(g.gemm_bytes(activation_form(g.M)) / (gm * 1e-3) / 1e9, 1),
-            "roofline": roofline_obj(g, gm, peaks, peaks_kind)})
+            "roofline": roofline_obj(g, gm, peaks, peaks_kind, int8_peak=int8_peak)})
     for m in (2048, 16):
         line = chain_line(apex, torch, m, steps, args.warmup, world)
         lines.append(line)

@@ -26,7 +26,7 @@ __all__ = [
     "quantize_act_expanded",
     "apex_w4a4_gemm_workspace_size", "apex_w4a4_group_partials", "apex_get_device_status",
     "apex_set_wait_limit_ns", "apex_status_string", "apex_debug_withhold_step",
-    "apex_debug_trace_next_gemm", "apex_debug_gemm_plan",
+    "apex_debug_trace_next_gemm", "apex_debug_gemm_plan", "apex_debug_partials_split",
     "pack_weights", "quantize_act", "gemm", "workspace",
 ]
 
@@ -100,6 +100,8 @@ def load_library(build_if_missing: bool = True):
         lib.apex_status_string.restype = ctypes.c_char_p
         lib.apex_debug_withhold_step.argtypes = [I32]
         lib.apex_debug_withhold_step.restype = None
+        lib.apex_debug_partials_split.argtypes = [I32]
+        lib.apex_debug_partials_split.restype = None
         lib.apex_debug_trace_next_gemm.argtypes = [P, I32, I32]
         lib.apex_debug_trace_next_gemm.restype = None
         lib.apex_debug_gemm_plan.argtypes = [I64, I64, I64, I32, I32, P]
@@ -267,6 +269,10 @@ def apex_set_wait_limit_ns(ns: int):
 
 def apex_debug_withhold_step(step: int):
     load_library().apex_debug_withhold_step(int(step))
+
+
+def apex_debug_partials_split(on: bool):
+    load_library().apex_debug_partials_split(1 if on else 0)
 
 
 def apex_debug_trace_next_gemm(trace, ctas: int, steps: int):

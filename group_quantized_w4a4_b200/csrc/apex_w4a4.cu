@@ -12,6 +12,7 @@
 
 #include "apex_w4a4.h"
 #include "gemm.cuh"
+#include "gemm_f8.cuh"
 #include "ptx.cuh"
 #include "quantize.cuh"
 
@@ -22,6 +23,7 @@ using apex::GemmCfg;
 
 uint64_t g_wait_limit_ns = 2000000000ull;
 thread_local int t_withhold = -1;
+thread_local int t_partials_split = 0;
 thread_local unsigned long long* t_trace = nullptr;
 thread_local int t_trace_ctas = 0;
 thread_local int t_trace_steps = 0;
@@ -318,10 +320,11 @@ void attach_workspace(const Plan& p, GemmArgs& a, void* ws) {
 }
 
 apex_status_t quantize_launch(const void* x, int64_t rows, int64_t K, int32_t group, void* packed,
-                              void* scales, void* stream, bool expanded = false) {
+                              void* scales, void* stream, bool expanded = false,
+                              bool e4m3 = false) {
   if (!x || !packed || !scales) return APEX_ERR_INVALID_ARG;
   if (rows <= 0 || K <= 0 || group <= 0 || K % group || group % 128) return APEX_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(packed, expanded ? 8 : 4) || !aligned(scales, 2))
+  if (!aligned(x, 16) || !aligned(packed, (expanded || e4m3) ? 8 : 4) || !aligned(scales, 2))
     return APEX_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t units = rows * (K / group);
@@ -338,10 +341,20 @@ apex_status_t quantize_launch(const void* x, int64_t rows, int64_t K, int32_t gr
   __half* sc = static_cast<__half*>(scales);
   const unsigned nb = (unsigned)blocks;
   cudaError_t e;
-  if (expanded) {
+  if (e4m3) {
+    if (group == 128)
+      e = launch_pdl(apex::quantize_pack_kernel<1, apex::FORM_E4M3>, nb, threads, 0, s, xh, rows,
+                     K, group, pk, sc);
+    else if (group == 512)
+      e = launch_pdl(apex::quantize_pack_kernel<4, apex::FORM_E4M3>, nb, threads, 0, s, xh, rows,
+                     K, group, pk, sc);
+    else
+      e = launch_pdl(apex::quantize_pack_kernel<0, apex::FORM_E4M3>, nb, threads, 0, s, xh, rows,
+                     K, group, pk, sc);
+  } else if (expanded) {
     if (group != 128) return APEX_ERR_UNSUPPORTED;
-    e = launch_pdl(apex::quantize_pack_kernel<1, true>, nb, threads, 0, s, xh, rows, K, group,
-                   pk, sc);
+    e = launch_pdl(apex::quantize_pack_kernel<1, apex::FORM_EXPANDED>, nb, threads, 0, s, xh,
+                   rows, K, group, pk, sc);
   } else if (group == 128) {
     e = launch_pdl(apex::quantize_pack_kernel<1>, nb, threads, 0, s, xh, rows, K, group, pk, sc);
   } else if (group == 256) {
@@ -418,9 +431,137 @@ apex_status_t gemm_entry(bool a_expanded, int64_t M, int64_t N, int64_t K, int32
                     : launch_gemm<apex::MODE_PACKED>(p, maps, a, s);
 }
 
+// ------------------------------------------------------------------ the E4M3-carrier GEMM
+
+struct F8Plan {
+  int tiles_m = 0, tiles_n = 0, T = 0, P = 0;
+};
+
+F8Plan make_f8_plan(int64_t M, int64_t N, int sms_override = 0) {
+  F8Plan p;
+  p.tiles_m = (int)((M + 127) / 128);
+  p.tiles_n = (int)((N + 255) / 256);
+  p.T = p.tiles_m * p.tiles_n;
+  const int sms = sms_override > 0 ? sms_override : dev_info().sms;
+  p.P = p.T < sms ? p.T : sms;
+  return p;
+}
+
+template <bool DUMP>
+apex_status_t launch_f8(const F8Plan& p, const CUtensorMap& ma, const CUtensorMap& mb,
+                        const apex::F8Args& a, cudaStream_t s) {
+  using C = apex::F8Cfg<DUMP>;
+  auto kern = apex::w4a4_gemm_f8_kernel<DUMP>;
+  static thread_local int attr_dev = -1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return APEX_ERR_CUDA;
+  if (attr_dev != dev) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+        cudaSuccess)
+      return APEX_ERR_CUDA;
+    attr_dev = dev;
+  }
+  return cuda_status(launch_pdl(kern, (unsigned)p.P, C::THREADS, (size_t)C::SMEM, s, ma, mb, a));
+}
+
+// The shared part of apex_w4a4_gemm_fp8 and the partials export: checks, plan, maps.
+apex_status_t f8_setup(int64_t M, int64_t N, int64_t K, int32_t group_w, const void* a_codes,
+                       const void* w_codes, F8Plan& p, apex::F8Args& a, CUtensorMap& ma,
+                       CUtensorMap& mb) {
+  if (!a_codes || !w_codes) return APEX_ERR_INVALID_ARG;
+  if (!aligned(a_codes, 16) || !aligned(w_codes, 16)) return APEX_ERR_ALIGNMENT;
+  p = make_f8_plan(M, N);
+  memset(&a, 0, sizeof(a));
+  a.M = (int)M;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.G = (int)(K / 128);
+  a.Gw = (int)(K / group_w);
+  a.gpg = group_w / 128;
+  a.tiles_m = p.tiles_m;
+  a.tiles_n = p.tiles_n;
+  a.T = p.T;
+  a.P = p.P;
+  a.wait_ns = g_wait_limit_ns;
+  memset(&ma, 0, sizeof(ma));
+  memset(&mb, 0, sizeof(mb));
+  if (!make_expanded_map(&ma, a_codes, M, K, 128) || !make_expanded_map(&mb, w_codes, N, K, 256))
+    return APEX_ERR_CUDA;
+  return APEX_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+apex_status_t apex_quantize_act_int4_fp8(const void* x_f16, int64_t M, int64_t K,
+                                         int32_t group_a, void* x_codes, void* x_scales_f16,
+                                         void* stream) {
+  if (group_a != 128 && group_a > 0 && K % group_a == 0 && group_a % 128 == 0)
+    return APEX_ERR_UNSUPPORTED;
+  return quantize_launch(x_f16, M, K, group_a, x_codes, x_scales_f16, stream, false, true);
+}
+
+apex_status_t apex_pack_weights_int4_fp8(const void* w_f16, int64_t N, int64_t K,
+                                         int32_t group_w, void* w_codes, void* w_scales_f16,
+                                         void* stream) {
+  return quantize_launch(w_f16, N, K, group_w, w_codes, w_scales_f16, stream, false, true);
+}
+
+apex_status_t apex_unpack_int4_fp8(const void* packed, int64_t rows, int64_t K, void* codes,
+                                   void* stream) {
+  if (!packed || !codes) return APEX_ERR_INVALID_ARG;
+  if (rows <= 0 || K <= 0 || K % 16) return APEX_ERR_INVALID_ARG;
+  if (!aligned(packed, 8) || !aligned(codes, 16)) return APEX_ERR_ALIGNMENT;
+  const int64_t words = rows * (K / 16);   // 8 packed bytes -> 16 codes each
+  int64_t blocks = (words + 255) / 256;
+  const int64_t cap = (int64_t)dev_info().sms * 8;
+  if (blocks > cap) blocks = cap;
+  cudaError_t e = launch_pdl(apex::unpack_e4m3_kernel, (unsigned)blocks, 256, 0,
+                             static_cast<cudaStream_t>(stream),
+                             static_cast<const uint8_t*>(packed), words,
+                             static_cast<uint8_t*>(codes));
+  if (e != cudaSuccess) return APEX_ERR_CUDA;
+  return cuda_status(cudaPeekAtLastError());
+}
+
+apex_status_t apex_w4a4_gemm_fp8(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                 int32_t group_w, const void* a_codes, const void* a_scales,
+                                 const void* w_codes, const void* w_scales, void* y_f16,
+                                 void* stream) {
+  apex_status_t st = check_gemm_args(M, N, K, group_a, group_w);
+  if (st != APEX_OK) return st;
+  if (!a_scales || !w_scales || !y_f16) return APEX_ERR_INVALID_ARG;
+  if (!aligned(a_scales, 2) || !aligned(w_scales, 2) || !aligned(y_f16, 2))
+    return APEX_ERR_ALIGNMENT;
+  F8Plan p;
+  apex::F8Args a;
+  CUtensorMap ma, mb;
+  st = f8_setup(M, N, K, group_w, a_codes, w_codes, p, a, ma, mb);
+  if (st != APEX_OK) return st;
+  a.sa = static_cast<const __half*>(a_scales);
+  a.sw = static_cast<const __half*>(w_scales);
+  a.y = static_cast<__half*>(y_f16);
+  a.sa_vec = a.G % 8 == 0 && aligned(a_scales, 16);
+  a.y_vec = N % 8 == 0 && aligned(y_f16, 16);
+  return launch_f8<false>(p, ma, mb, a, static_cast<cudaStream_t>(stream));
+}
+
+apex_status_t apex_w4a4_group_partials_fp8(int64_t M, int64_t N, int64_t K, const void* a_codes,
+                                           const void* w_codes, int32_t* partials_i32,
+                                           void* stream) {
+  apex_status_t st = check_gemm_args(M, N, K, 128, 128);
+  if (st != APEX_OK) return st;
+  if (!partials_i32) return APEX_ERR_INVALID_ARG;
+  if (!aligned(partials_i32, 4)) return APEX_ERR_ALIGNMENT;
+  F8Plan p;
+  apex::F8Args a;
+  CUtensorMap ma, mb;
+  st = f8_setup(M, N, K, 128, a_codes, w_codes, p, a, ma, mb);
+  if (st != APEX_OK) return st;
+  a.dump = partials_i32;
+  return launch_f8<true>(p, ma, mb, a, static_cast<cudaStream_t>(stream));
+}
 
 apex_status_t apex_pack_weights_int4(const void* w_f16, int64_t N, int64_t K, int32_t group_w,
                                      void* w_packed_u8, void* w_scales_f16, void* stream) {
@@ -536,7 +677,8 @@ static __device__ __align__(256) uint8_t g_static_scratch[APEX_STATIC_SCRATCH_BY
 namespace {
 
 // Device address of g_static_scratch, looked up once per device (with that device current)
-// on the first call there.  The array's host-side name is only a handle, never an address.
+// on the first call there, and kept until the process exits (a device reset afterwards is
+// not supported).  The array's host-side name is only a handle, never an address.
 apex_status_t static_scratch_ptr(void** out) {
   static std::mutex mu;
   static void* ptrs[64] = {};
@@ -569,6 +711,8 @@ apex_status_t apex_w4a4_gemm_noalloc(int64_t M, int64_t N, int64_t K, int32_t gr
   // The problem's stream-K scratch must fit the fixed array; larger problems are refused.
   if (workspace_for(p) > (size_t)APEX_STATIC_SCRATCH_BYTES) return APEX_ERR_UNSUPPORTED;
   GemmArgs a = base_args(p, M, N, K, group_w, a_scales, w_scales, y_f16);
+  a.withhold = t_withhold;   // test hook, as in apex_w4a4_gemm
+  t_withhold = -1;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (p.streamk) {
     void* scratch = nullptr;
@@ -594,8 +738,13 @@ apex_status_t apex_w4a4_group_partials(int64_t M, int64_t N, int64_t K, const vo
   if (!a_packed || !w_packed || !partials_i32) return APEX_ERR_INVALID_ARG;
   if (!aligned(a_packed, 16) || !aligned(w_packed, 16) || !aligned(partials_i32, 4))
     return APEX_ERR_ALIGNMENT;
-  Plan p = make_plan(M, N, K, false);
+  // The work plan: whole tiles, or (test hook) the split plan apex_w4a4_gemm takes with a
+  // workspace -- each (tile, K-group) is still handled by exactly one CTA, which stores its
+  // partial, so no scratch is needed and the split parts are never added.
+  Plan p = make_plan(M, N, K, t_partials_split != 0);
+  t_partials_split = 0;
   GemmArgs a = base_args(p, M, N, K, 128, nullptr, nullptr, nullptr);
+  a.cluster = 1;
   a.dump = partials_i32;
   Maps maps;
   memset(&maps, 0, sizeof(maps));
@@ -636,6 +785,8 @@ apex_status_t apex_debug_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t sms,
 }
 
 void apex_debug_withhold_step(int32_t step) { t_withhold = step; }
+
+void apex_debug_partials_split(int32_t on) { t_partials_split = on ? 1 : 0; }
 
 void apex_debug_trace_next_gemm(uint64_t* trace, int32_t ctas, int32_t steps) {
   t_trace = reinterpret_cast<unsigned long long*>(trace);

@@ -724,27 +724,27 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE, QOUT>::THREADS, 1)
 #pragma unroll
         for (int o = 1; o < TPT; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
         const __half sc = group_scale(am);
-        const float sf = __half2float(sc);
+        const QScale qs = make_qscale(__half2float(sc));
         const int m = m0t + tok;
         if (m < M) {
           if (args.qexp) {
             uint8_t* dst = args.qout + (size_t)m * N + n0t + part * RPT;
 #pragma unroll
             for (int j = 0; j < R8; j += 2) {
-              const uint2 x0 = quant_expand8(v[j], sf), x1 = quant_expand8(v[j + 1], sf);
+              const uint2 x0 = quant_expand8(v[j], qs), x1 = quant_expand8(v[j + 1], qs);
               *reinterpret_cast<uint4*>(dst + 8 * j) = make_uint4(x0.x, x0.y, x1.x, x1.y);
             }
           } else {
             uint8_t* dst = args.qout + (size_t)m * (N / 2) + n0t / 2 + part * (RPT / 2);
             if constexpr (R8 == 2) {
               *reinterpret_cast<uint2*>(dst) =
-                  make_uint2(quant_pack8(v[0], sf), quant_pack8(v[1], sf));
+                  make_uint2(quant_pack8(v[0], qs), quant_pack8(v[1], qs));
             } else {
 #pragma unroll
               for (int j = 0; j < R8; j += 4)
                 *reinterpret_cast<uint4*>(dst + 4 * j) =
-                    make_uint4(quant_pack8(v[j], sf), quant_pack8(v[j + 1], sf),
-                               quant_pack8(v[j + 2], sf), quant_pack8(v[j + 3], sf));
+                    make_uint4(quant_pack8(v[j], qs), quant_pack8(v[j + 1], qs),
+                               quant_pack8(v[j + 2], qs), quant_pack8(v[j + 3], qs));
             }
           }
           if (part == 0) args.qscale[(size_t)m * (N / 128) + n0t / 128] = sc;

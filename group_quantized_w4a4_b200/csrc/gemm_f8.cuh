@@ -1,0 +1,437 @@
+// gemm_f8.cuh -- the W4A4 GEMM for compute-bound shapes (many tokens), with the 4-bit
+// values carried as E4M3 codes so that the tensor core returns every group's exact integer
+// partial already in fp32.
+//
+// The method ("APEX4: Efficient Pure W4A4 LLM Inference via Intra-SM Compute Rebalancing",
+// abstract) multiplies 4-bit integers on the tensor cores and dequantises each 128-wide
+// K-group's integer partial on the CUDA cores:
+//   Y[m,n] = sum_g P_g[m,n] * sa[m,g] * sw[n, g*128/gw],  P_g = sum_{k in g} qa[m,k]*qw[n,k].
+// On B200 the per-group dequantisation, not the MMA, limits this (the abstract's "group
+// dequantization overhead" on the CUDA cores; B200's tensor : CUDA-core throughput ratio is
+// A100-like).  An int8 MMA leaves an int32 partial that costs an int->fp32 conversion per
+// partial on top of the scale arithmetic.  Every q in [-8, 7] is an E4M3 value, and so is
+// every product (|qa*qw| <= 64); a group's sum of 128 such products is an integer of at most
+// 2^13 in magnitude, which the fp32 accumulator of kind::f8f6f4 holds exactly.  So with the
+// operands stored as E4M3 codes of q (one byte per element, written by the quantizer), the
+// MMA gives the same exact P_g as an int8 MMA, as an fp32 value, and the epilogue only
+// multiplies and adds.  (Exactness is checked bit for bit against the oracle's int64
+// partials by the partials export of this kernel.)
+//
+// Tile: 128 tokens (tensor-memory lanes, MMA M) x 256 weight rows (MMA N), one K-group per
+// pipeline stage: a [128 x 128 B] token box and a [256 x 128 B] weight box, both by TMA with
+// 128-byte swizzle into a 4-deep ring.  Per K-group, 4 MMAs (K = 32 each) write the group's
+// partial into one of two 256-column tensor-memory slots, so the epilogue drains one slot
+// while the next group's MMAs fill the other.
+// Roles (384 threads in three warpgroups, one persistent CTA per SM, whole tiles
+// round-robin):
+//   warp 0       TMA producer (lane 0 issues)
+//   warp 1       MMA issuer (lane 0 issues; commits free the stage and fill the slot)
+//   warps 2, 3   idle (they only complete the first warpgroup)
+//   warps 4..11  epilogue: warp w reads tensor-memory lanes 32*(w%4)..+31 (one token each)
+//                and columns 128*((w-4)/4)..+127 of the slot; per group and column:
+//                s = sa*sw (fp32, exact), acc += P*s (packed f32x2 math).
+// The block launches with 168 registers a thread (three warps per SM sub-partition); the
+// first warpgroup then gives up all but 40 and the two epilogue warpgroups take 232, which
+// their 128 accumulators and two 32-column partial loads in flight need.
+// Weight scales are staged in shared memory as fp32 [8 groups][256 columns] per block of 8
+// K-groups, two blocks (the next one is loaded while the current one is used); each
+// epilogue thread keeps its token's scales in registers, also one block ahead.
+#pragma once
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+
+namespace apex {
+
+struct F8Args {
+  int M, N, K;
+  int G;             // K / 128
+  int Gw;            // K / gw
+  int gpg;           // K-groups per weight scale (gw / 128)
+  int tiles_m, tiles_n, T;
+  int P;             // persistent CTAs (gridDim.x)
+  int sa_vec;        // sa rows readable as 16-byte blocks of 8 groups
+  int sw_vec;        // sw rows readable as 16-byte blocks of 8 groups (gw == 128)
+  int y_vec;         // Y rows writable as 16-byte vectors
+  const __half* sa;  // [M][G]
+  const __half* sw;  // [N][Gw]
+  __half* y;         // [M][N]
+  int32_t* dump;     // [G][M][N] per-group partials (export kernel only)
+  unsigned long long wait_ns;
+};
+
+template <bool DUMP>
+struct F8Cfg {
+  static constexpr int BM = 128;                   // tokens per tile
+  static constexpr int BN = 256;                   // weight rows per tile
+  static constexpr int NS = 4;                     // operand stages, one K-group each
+  static constexpr int A_BYTES = BM * 128;
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int STAGE = A_BYTES + B_BYTES;  // 48 KB
+  static constexpr int SLOTS = 2;                  // partial slots of BN columns
+  static constexpr int TMEM_COLS = SLOTS * BN;     // 512
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int EPI_THREADS = EPI_WARPS * 32;
+  static constexpr int THREADS = 128 + EPI_THREADS;  // 384
+  static constexpr int REGS_LAUNCH = 168;          // 3 warps x 32 x 168 <= 16384 per quarter
+  static constexpr int REGS_CTRL = 40;
+  static constexpr int REGS_EPI = 232;
+  static_assert(128 * REGS_CTRL + EPI_THREADS * REGS_EPI <= THREADS * REGS_LAUNCH,
+                "register budgets fit the block's pool");
+  static constexpr int CPT = BN / 2;               // columns per epilogue thread (128)
+  static constexpr int SWB = 8 * BN * 4;           // one staged block of weight scales (fp32)
+  static constexpr int OFF_STAGE = 0;
+  static constexpr int OFF_SW = NS * STAGE;
+  static constexpr int OFF_BAR = OFF_SW + 2 * SWB;
+  static constexpr int NBAR = 2 * NS + 2 * SLOTS + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;   // + alignment slack
+  static_assert(STAGE % 1024 == 0 && A_BYTES % 1024 == 0, "swizzle atoms stay aligned");
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(TMEM_COLS <= 512, "tensor memory budget");
+};
+
+// Tile t -> (token tile, weight tile): bands of 8 token tiles, weight tiles across each band,
+// so the CTAs running at once share both operands' tiles in L2.
+__device__ __forceinline__ void f8_tile(const F8Args& a, int t, int& tm, int& tn) {
+  constexpr int BAND = 8;
+  const int per = BAND * a.tiles_n;
+  const int band = t / per;
+  const int first = band * BAND;
+  const int rows = min(a.tiles_m - first, BAND);
+  const int r = t - band * per;
+  tm = first + r % rows;
+  tn = r / rows;
+}
+
+// The 8 fp16 scales of groups gb8 .. gb8+7 of one row (raw bits, zeros outside [0, G) and
+// for rows outside the matrix): one 16-byte load when `vec` (8 consecutive scale groups,
+// 16-byte aligned), else one load per group; gpg = K-groups per scale group.
+__device__ __forceinline__ uint4 scale_block8(const __half* base, int row, int rows, int ld,
+                                              int gb8, int G, int gpg, bool vec) {
+  if (row >= rows) return make_uint4(0, 0, 0, 0);
+  const __half* r = base + (size_t)row * ld;
+  if (vec) return __ldg(reinterpret_cast<const uint4*>(r + gb8));
+  uint32_t h[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    h[j] = gb8 + j < G ? (uint32_t)__half_as_ushort(r[(gb8 + j) / gpg]) : 0u;
+  return make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
+                    h[6] | (h[7] << 16));
+}
+
+__device__ __forceinline__ float half_at(const uint4& v, int j) {
+  const uint32_t w = j < 2 ? v.x : j < 4 ? v.y : j < 6 ? v.z : v.w;
+  return __half2float(__ushort_as_half((uint16_t)((j & 1) ? (w >> 16) : (w & 0xFFFFu))));
+}
+
+__device__ __forceinline__ uint32_t half2_bits(float2 v) {
+  const __half2 h = __float22half2_rn(v);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+
+template <bool DUMP>
+__global__ void __launch_bounds__(F8Cfg<DUMP>::THREADS, 1)
+    __maxnreg__(F8Cfg<DUMP>::REGS_LAUNCH) w4a4_gemm_f8_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const F8Args args) {
+  using C = F8Cfg<DUMP>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* stages = smem + C::OFF_STAGE;
+  float* s_sw = reinterpret_cast<float*>(smem + C::OFF_SW);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* full = bars;                 // stage loaded (TMA bytes)
+  uint64_t* empty = full + C::NS;        // stage read by its MMAs (commit)
+  uint64_t* tfull = empty + C::NS;       // slot holds a finished partial (commit)
+  uint64_t* tempty = tfull + C::SLOTS;   // slot read out (one arrival per epilogue warp)
+  uint64_t* mma_done = tempty + C::SLOTS;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  int* s_abort = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
+  int* s_never = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint64_t lim = args.wait_ns;
+  const int G = args.G;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NS; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    for (int i = 0; i < C::SLOTS; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), C::EPI_WARPS);
+    }
+    mbar_init(smem_u32(mma_done), 1);
+    *s_abort = 0;
+    *s_never = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(s_tmem), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // launched as a programmatic dependent: the prologue above overlaps the previous grid's
+  // tail; the roles that touch global memory wait for it below
+  grid_dep_launch();
+  const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(s_tmem);
+  volatile int* abort_flag = s_abort;
+  volatile int* never = s_never;
+  if (warp < 4)
+    regs_dec<C::REGS_CTRL>();
+  else
+    regs_inc<C::REGS_EPI>();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    grid_dep_wait();
+    int it = 0, last = -1;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < args.T; t += args.P) {
+      int tm, tn;
+      f8_tile(args, t, tm, tn);
+      for (int g = 0; g < G; ++g, ++it) {
+        const int st = it % C::NS;
+        ok = mbar_wait(smem_u32(&empty[st]), ((uint32_t)(it / C::NS) & 1u) ^ 1u, lim, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        if (lane == 0) {
+          const uint32_t fb = smem_u32(&full[st]);
+          uint8_t* sa_dst = stages + st * C::STAGE;
+          mbar_arrive_expect_tx(fb, C::STAGE);
+          tma_load_2d(smem_u32(sa_dst), &tmA, fb, g * 128, tm * C::BM);
+          tma_load_2d(smem_u32(sa_dst + C::A_BYTES), &tmB, fb, g * 128, tn * C::BN);
+        }
+        __syncwarp();
+        last = it;
+      }
+    }
+    // never leave the CTA with bulk copies in flight
+    for (int s = (last - C::NS + 1 > 0 ? last - C::NS + 1 : 0); s <= last; ++s)
+      mbar_wait(smem_u32(&full[s % C::NS]), (uint32_t)(s / C::NS) & 1u, lim, never);
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc = idesc_e4m3(C::BM, C::BN);
+    int it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < args.T; t += args.P) {
+      for (int g = 0; g < G; ++g, ++it) {
+        const int st = it % C::NS, sl = it % C::SLOTS;
+        ok = mbar_wait2(smem_u32(&full[st]), (uint32_t)(it / C::NS) & 1u,
+                        smem_u32(&tempty[sl]), ((uint32_t)(it / C::SLOTS) & 1u) ^ 1u, lim,
+                        abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint64_t a0 = smem_desc_k_sw128(smem_u32(stages + st * C::STAGE));
+          const uint64_t b0 = smem_desc_k_sw128(smem_u32(stages + st * C::STAGE + C::A_BYTES));
+          const uint32_t d = tbase + sl * C::BN;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)   // K = 32 bytes per MMA: +2 in 16-byte descriptor units
+            umma_f8_ss(d, a0 + (uint64_t)(2 * j), b0 + (uint64_t)(2 * j), idesc, j > 0 ? 1u : 0u);
+          umma_commit(smem_u32(&empty[st]));
+          umma_commit(smem_u32(&tfull[sl]));
+        }
+        __syncwarp();
+      }
+    }
+    if (lane == 0) umma_commit(smem_u32(mma_done));
+    __syncwarp();
+    mbar_wait(smem_u32(mma_done), 0u, lim, never);
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    grid_dep_wait();   // scales and outputs are global memory
+    const int ew = warp - 4;                    // 0..7
+    const int et = threadIdx.x - 128;           // 0..255: the weight column it stages
+    const int lq = warp & 3;                    // tensor-memory lane quarter of this warp
+    const int ch = ew >> 2;                     // column half: columns 128*ch .. +127
+    const int row = 32 * lq + lane;             // token of the tile
+    const uint32_t t_lane = (uint32_t)(32 * lq) << 16;
+    constexpr uint32_t EB = 1;                  // named barrier of the epilogue warps
+    const bool sa_vec = args.sa_vec != 0, sw_vec = args.sw_vec != 0;
+    float2 acc[C::CPT / 2];
+    bool ok = true, aborted = false;
+    int it = 0;
+    int b = 0;   // flat 8-group block counter: its weight scales are staged in s_sw[b & 1]
+
+    // weight scales of one block: thread et stages column et, all 8 groups
+    auto stage_sw = [&](float* blk, const uint4& v) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) blk[j * C::BN + et] = half_at(v, j);
+    };
+    // the first block's scales before the first group
+    int t = blockIdx.x;
+    uint4 sa_c = make_uint4(0, 0, 0, 0);
+    if (t < args.T && !DUMP) {
+      int tm, tn;
+      f8_tile(args, t, tm, tn);
+      stage_sw(s_sw, scale_block8(args.sw, tn * C::BN + et, args.N, args.Gw, 0, G, args.gpg,
+                                  sw_vec));
+      sa_c = scale_block8(args.sa, tm * C::BM + row, args.M, G, 0, G, 1, sa_vec);
+    }
+    aborted = bar_red_or(EB, C::EPI_THREADS, false);
+    for (; !aborted && t < args.T; t += args.P) {
+      int tm, tn;
+      f8_tile(args, t, tm, tn);
+      const int m = tm * C::BM + row;
+      const int n0 = tn * C::BN + ch * C::CPT;
+#pragma unroll
+      for (int e = 0; e < C::CPT / 2; ++e) acc[e] = make_float2(0.0f, 0.0f);
+      for (int gb8 = 0; gb8 < G; gb8 += 8, ++b) {
+        // the next block's scales (of this tile, or the first of the next) are in flight
+        // while this block is processed
+        const bool more = gb8 + 8 < G;
+        int ntm = tm, ntn = tn;
+        if (!more && t + args.P < args.T) f8_tile(args, t + args.P, ntm, ntn);
+        const bool have_next = !DUMP && (more || t + args.P < args.T);
+        const int ngb = more ? gb8 + 8 : 0;
+        uint4 sw_n = make_uint4(0, 0, 0, 0), sa_n = make_uint4(0, 0, 0, 0);
+        if (have_next) {
+          sw_n = scale_block8(args.sw, ntn * C::BN + et, args.N, args.Gw, ngb, G, args.gpg,
+                              sw_vec);
+          sa_n = scale_block8(args.sa, ntm * C::BM + row, args.M, G, ngb, G, 1, sa_vec);
+        }
+        const float* swb = s_sw + (b & 1) * (C::SWB / 4) + ch * C::CPT;
+        const int je = min(8, G - gb8);
+        for (int j = 0; j < je && ok; ++j, ++it) {
+          const int sl = it % C::SLOTS;
+          ok = mbar_wait(smem_u32(&tfull[sl]), (uint32_t)(it / C::SLOTS) & 1u, lim, abort_flag);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t td = tbase + t_lane + sl * C::BN + ch * C::CPT;
+          const float saf = half_at(sa_c, j);
+          const float2 sa2 = make_float2(saf, saf);
+          const float* swj = swb + j * C::BN;
+          // four 32-column loads, the next one in flight while the current one is used
+          uint32_t p[2][32];
+          tmem_ld32_nowait(td, p[0]);
+          tmem_ld_wait32(p[0]);
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t* pc = p[cc & 1];
+            if (cc < 3) tmem_ld32_nowait(td + 32 * (cc + 1), p[(cc + 1) & 1]);
+            if constexpr (DUMP) {
+              int32_t* dst = args.dump + ((size_t)(gb8 + j) * args.M + m) * args.N + n0 + cc * 32;
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (m < args.M && n0 + cc * 32 + e < args.N)
+                  dst[e] = __float2int_rn(__uint_as_float(pc[e]));
+            } else {
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const float4 s4 = *reinterpret_cast<const float4*>(swj + cc * 32 + 4 * q);
+                const float2 s_a = __fmul2_rn(make_float2(s4.x, s4.y), sa2);
+                const float2 s_b = __fmul2_rn(make_float2(s4.z, s4.w), sa2);
+                acc[cc * 16 + 2 * q] = __ffma2_rn(
+                    make_float2(__uint_as_float(pc[4 * q]), __uint_as_float(pc[4 * q + 1])),
+                    s_a, acc[cc * 16 + 2 * q]);
+                acc[cc * 16 + 2 * q + 1] = __ffma2_rn(
+                    make_float2(__uint_as_float(pc[4 * q + 2]), __uint_as_float(pc[4 * q + 3])),
+                    s_b, acc[cc * 16 + 2 * q + 1]);
+              }
+            }
+            if (cc < 3) tmem_ld_wait32(p[(cc + 1) & 1]);
+            if (cc == 2) {
+              // every load of the slot has completed: hand it back to the MMA
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(smem_u32(&tempty[sl]));
+            }
+          }
+        }
+        // the next block's weight scales into the other buffer; one barrier per block (also
+        // the epilogue's one decision to give up, so no warp is left waiting here)
+        if (have_next) stage_sw(s_sw + ((b + 1) & 1) * (C::SWB / 4), sw_n);
+        aborted = bar_red_or(EB, C::EPI_THREADS, !ok);
+        if (aborted) break;
+        sa_c = sa_n;
+      }
+      if (aborted) break;
+      if constexpr (!DUMP) {
+        // the finished tile: this thread's token row, 128 consecutive outputs
+        if (m < args.M) {
+          __half* dst = args.y + (size_t)m * args.N + n0;
+          if (args.y_vec && n0 + C::CPT <= args.N) {
+#pragma unroll
+            for (int e = 0; e < C::CPT / 2; e += 4)
+              *reinterpret_cast<uint4*>(dst + 2 * e) =
+                  make_uint4(half2_bits(acc[e]), half2_bits(acc[e + 1]), half2_bits(acc[e + 2]),
+                             half2_bits(acc[e + 3]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < C::CPT; ++e) {
+              const float v = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
+              if (n0 + e < args.N) dst[e] = __float2half_rn(v);
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+// Packed int4 [rows][K/2] -> E4M3 codes of the same q [rows][K] (element order).  Each thread
+// turns 8 packed bytes into 16 codes with byte-permute table lookups: the codes of q = 0..7
+// and of q = -8..-1 are two 8-byte tables, a nibble's low three bits index both and its sign
+// bit picks one.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// E4M3 codes of the four nibbles in the low 16 bits of w (nibble i -> byte i).
+__device__ __forceinline__ uint32_t e4m3_of_nibbles(uint32_t w) {
+  // E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits) of 0..7 and of -8..-1
+  constexpr uint32_t P0 = 0x44403800u, P1 = 0x4E4C4A48u;   // 0, 1, 2, 3 | 4, 5, 6, 7
+  constexpr uint32_t N0 = 0xCACCCED0u, N1 = 0xB8C0C4C8u;   // -8,-7,-6,-5 | -4,-3,-2,-1
+  const uint32_t idx = w & 0x7777u;
+  const uint32_t pos = prmt(P0, P1, idx);
+  const uint32_t neg = prmt(N0, N1, idx);
+  // 0xFF in byte i where nibble i is negative: selector 0xC (sign of byte 4 = 0x80) or 0x0
+  const uint32_t s = w & 0x8888u;
+  const uint32_t mask = prmt(0u, 0x80u, s | (s >> 1));
+  return (neg & mask) | (pos & ~mask);
+}
+
+__global__ void __launch_bounds__(256) unpack_e4m3_kernel(const uint8_t* __restrict__ packed,
+                                                         int64_t words, uint8_t* __restrict__ codes) {
+  grid_dep_wait();
+  grid_dep_launch();
+  // one unit = 8 packed bytes (16 elements) -> 16 codes
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < words;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const uint2 w = __ldg(reinterpret_cast<const uint2*>(packed) + i);
+    uint4 o;
+    o.x = e4m3_of_nibbles(w.x);
+    o.y = e4m3_of_nibbles(w.x >> 16);
+    o.z = e4m3_of_nibbles(w.y);
+    o.w = e4m3_of_nibbles(w.y >> 16);
+    reinterpret_cast<uint4*>(codes)[i] = o;
+  }
+}
+
+}  // namespace apex

@@ -34,23 +34,70 @@ __device__ __forceinline__ __half group_scale(float absmax) {
   return __float2half_rn(__fdiv_rn(absmax, 7.0f));
 }
 
-// One value (an fp16 value widened to fp32) against scale sf (fp32 copy of the stored fp16
-// scale): clamp(round_half_even(f / sf), -8, 7), 0 when sf == 0.
-__device__ __forceinline__ int quant1(float f, float sf) {
-  if (sf == 0.0f) return 0;
-  const int q = __float2int_rn(__fdiv_rn(f, sf));
-  return min(max(q, -8), 7);
+// A group's stored scale in the form the per-value rule uses: s (fp32 copy of the stored
+// fp16 scale), r = 1/s correctly rounded, and s/2 (exact).
+struct QScale {
+  float s, r, h;
+};
+__device__ __forceinline__ QScale make_qscale(float sf) {
+  QScale q;
+  q.s = sf;
+  q.r = sf != 0.0f ? __frcp_rn(sf) : 0.0f;
+  q.h = 0.5f * sf;
+  return q;
 }
 
-// Quantize 8 fp16 values against scale sf and pack them into 4 bytes (little-endian:
+// One value (an fp16 value widened to fp32): clamp(round_half_even(f / s), -8, 7), 0 when
+// s == 0, without a division.  q0 = rne(f * r) is within one of the answer; the residual
+// e = f - q0 * s is exact in fp32 for fp16 f and s (one fma), and it decides the last step:
+// |e| > s/2 moves q0 one toward e, |e| == s/2 is a tie and moves it only if q0 is odd.
+// This equals the correctly rounded quotient's rounding for every (f, s) the quantizer
+// meets, which a CPU test checks exhaustively.
+__device__ __forceinline__ float quant1f(float f, const QScale& qs) {
+  if (qs.s == 0.0f) return 0.0f;
+  const float q0 = rintf(__fmul_rn(f, qs.r));
+  const float e = __fmaf_rn(-q0, qs.s, f);
+  const float ae = fabsf(e);
+  const bool odd = (__float2int_rn(q0) & 1) != 0;
+  const float q = (ae > qs.h || (ae == qs.h && odd)) ? q0 + copysignf(1.0f, e) : q0;
+  return fminf(fmaxf(q, -8.0f), 7.0f);
+}
+
+__device__ __forceinline__ int quant1(float f, const QScale& qs) {
+  return __float2int_rn(quant1f(f, qs));
+}
+
+// Two integer-valued floats (|v| <= 8) as E4M3 codes, exact: lo in bits 0..7, hi in 8..15.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// The same 8 values as the E4M3 codes of q (one byte per element, in element order): the
+// 8-bit float operand form of the tensor cores' kind::f8f6f4, which holds every q in
+// [-8, 7] exactly.
+__device__ __forceinline__ uint2 quant_e4m3_8(const uint4& v, const QScale& qs) {
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
+  uint32_t w[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float2 a = __half22float2(h[2 * i]), b = __half22float2(h[2 * i + 1]);
+    w[i] = e4m3x2(quant1f(a.x, qs), quant1f(a.y, qs)) |
+           (e4m3x2(quant1f(b.x, qs), quant1f(b.y, qs)) << 16);
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+// Quantize 8 fp16 values against the group scale qs and pack them into 4 bytes (little-endian:
 // element 0 in the low nibble of byte 0).
-__device__ __forceinline__ uint32_t quant_pack8(const uint4& v, float sf) {
+__device__ __forceinline__ uint32_t quant_pack8(const uint4& v, const QScale& qs) {
   const __half2* h = reinterpret_cast<const __half2*>(&v);
   uint32_t out = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float2 f = __half22float2(h[i]);
-    const int q0 = quant1(f.x, sf), q1 = quant1(f.y, sf);
+    const int q0 = quant1(f.x, qs), q1 = quant1(f.y, qs);
     out |= ((uint32_t)(q0 & 0xF) | ((uint32_t)(q1 & 0xF) << 4)) << (8 * i);
   }
   return out;
@@ -58,16 +105,31 @@ __device__ __forceinline__ uint32_t quant_pack8(const uint4& v, float sf) {
 
 // The same 8 values as 16*q in signed bytes, in the GEMM's operand order: bytes 0..3 hold
 // elements 0,2,4,6 and bytes 4..7 elements 1,3,5,7 (what the GEMM makes of a packed word).
-__device__ __forceinline__ uint2 quant_expand8(const uint4& v, float sf) {
-  const uint32_t w = quant_pack8(v, sf);
+__device__ __forceinline__ uint2 quant_expand8(const uint4& v, const QScale& qs) {
+  const uint32_t w = quant_pack8(v, qs);
   return make_uint2((w << 4) & 0xF0F0F0F0u, w & 0xF0F0F0F0u);
+}
+
+// Output forms of the quantizer: packed nibbles ([rows][K/2] bytes), the expanded int8
+// operand form ([rows][K] bytes of 16*q, see quant_expand8), or E4M3 codes of q ([rows][K]
+// bytes, element order, see quant_e4m3_8).
+enum QForm : int { FORM_PACKED = 0, FORM_EXPANDED = 1, FORM_E4M3 = 2 };
+
+template <int FORM>
+__device__ __forceinline__ void store_quantized(uint32_t* dst, uint2* xdst, const uint4& v,
+                                                const QScale& qs) {
+  if constexpr (FORM == FORM_EXPANDED)
+    *xdst = quant_expand8(v, qs);
+  else if constexpr (FORM == FORM_E4M3)
+    *xdst = quant_e4m3_8(v, qs);
+  else
+    *dst = quant_pack8(v, qs);
 }
 
 // CH > 0: the group is exactly CH 128-wide chunks, kept in registers (one pass over HBM).
 // CH == 0: any group width; absmax pass then quantize pass (the second pass hits L2).
-// EXP: write the expanded operand form ([rows][K] bytes of 16*q, see quant_expand8)
-// instead of packed nibbles ([rows][K/2] bytes).
-template <int CH, bool EXP = false>
+// FORM: the output form (QForm).
+template <int CH, int FORM = FORM_PACKED>
 __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __restrict__ x,
                                                             int64_t rows, int64_t K, int group,
                                                             uint8_t* __restrict__ packed,
@@ -107,15 +169,10 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __rest
       for (int off = 8; off >= 1; off >>= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
       const __half s = group_scale(amax);
-      const float sf = __half2float(s);
+      const QScale qs = make_qscale(__half2float(s));
       if (live) {
 #pragma unroll
-        for (int c = 0; c < CH; ++c) {
-          if constexpr (EXP)
-            xdst[c * 16] = quant_expand8(v[c], sf);
-          else
-            dst[c * 16] = quant_pack8(v[c], sf);
-        }
+        for (int c = 0; c < CH; ++c) store_quantized<FORM>(dst + c * 16, xdst + c * 16, v[c], qs);
         if (lane16 == 0) scales[row * G + g] = s;
       }
     } else {
@@ -127,14 +184,10 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __rest
       for (int off = 8; off >= 1; off >>= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
       const __half s = group_scale(amax);
-      const float sf = __half2float(s);
+      const QScale qs = make_qscale(__half2float(s));
       if (live) {
-        for (int c = 0; c < chunks; ++c) {
-          if constexpr (EXP)
-            xdst[c * 16] = quant_expand8(__ldg(src + c * 16), sf);
-          else
-            dst[c * 16] = quant_pack8(__ldg(src + c * 16), sf);
-        }
+        for (int c = 0; c < chunks; ++c)
+          store_quantized<FORM>(dst + c * 16, xdst + c * 16, __ldg(src + c * 16), qs);
         if (lane16 == 0) scales[row * G + g] = s;
       }
     }

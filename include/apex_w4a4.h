@@ -144,7 +144,9 @@ apex_status_t apex_w4a4_gemm_expanded_quant(int64_t M, int64_t N, int64_t K, int
  * calls no allocator.  A problem whose scratch would exceed that size is refused with
  * APEX_ERR_UNSUPPORTED.
  * The first call on each device looks the array's device address up (with that device
- * current), so make that first call before any stream capture.  All calls on a device
+ * current), so make that first call before any stream capture.  The address is kept for
+ * the rest of the process: resetting the device (cudaDeviceReset) or destroying and
+ * re-creating its primary context afterwards is not supported.  All calls on a device
  * share the one array and it keeps the previous call's contents (each call clears the
  * parts that must start at zero), so calls that overlap on the GPU -- on different
  * streams, or from different host threads -- race and must be ordered by the caller.
@@ -178,6 +180,70 @@ size_t apex_w4a4_linear_workspace_size(int64_t M, int64_t N, int64_t K, int32_t 
 /* Workspace bytes apex_w4a4_gemm would use for this problem (0 when it needs none). */
 size_t apex_w4a4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group_a,
                                      int32_t group_w);
+
+/*
+ * ---- The E4M3-carrier forms, for compute-bound shapes (many tokens).
+ *
+ * The same 4-bit values q, one byte per element in element order, each byte the E4M3 code
+ * of q (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; every q in [-8, 7] is an
+ * E4M3 value).  The tensor cores multiply such operands with an fp32 accumulator
+ * (kind::f8f6f4), which holds every group's integer partial exactly, so the GEMM below
+ * computes exactly what apex_w4a4_gemm computes while the per-group dequantisation needs
+ * no int-to-float conversion ("APEX4: Efficient Pure W4A4 LLM Inference via Intra-SM
+ * Compute Rebalancing", abstract: the group dequantisation on the CUDA cores is the
+ * bottleneck of the W4A4 GEMM).  Twice the bytes of the packed form: worth it where the
+ * math, not memory traffic, bounds the GEMM.
+ */
+
+/*
+ * Online activation quantization into E4M3 codes: the rule of apex_quantize_act_int4
+ * (group_a must be 128), x_codes [M][K] bytes (8-byte aligned; 16 for the GEMM), x_scales_f16
+ * [M][K/128] -- the same q and the same scales as the packed form.
+ */
+apex_status_t apex_quantize_act_int4_fp8(const void *x_f16, int64_t M, int64_t K,
+                                         int32_t group_a, void *x_codes, void *x_scales_f16,
+                                         void *stream);
+
+/*
+ * Offline weight quantization into E4M3 codes: the rule of apex_pack_weights_int4 (any
+ * group_w it accepts), w_codes [N][K] bytes (8-byte aligned; 16 for the GEMM), w_scales_f16
+ * [N][K/group_w] -- the same q and the same scales as the packed form.
+ */
+apex_status_t apex_pack_weights_int4_fp8(const void *w_f16, int64_t N, int64_t K,
+                                         int32_t group_w, void *w_codes, void *w_scales_f16,
+                                         void *stream);
+
+/*
+ * Packed int4 [rows][K/2] (the format of apex_pack_weights_int4) -> E4M3 codes of the same
+ * values [rows][K].  K % 16 == 0; packed 8-byte and codes 16-byte aligned.
+ */
+apex_status_t apex_unpack_int4_fp8(const void *packed, int64_t rows, int64_t K, void *codes,
+                                   void *stream);
+
+/*
+ * The W4A4 GEMM on E4M3-coded operands: y_f16 [M][N] = fp16_rne(sum_g P_g * sa * sw),
+ * accumulated in fp32, the same result rule as apex_w4a4_gemm.
+ *   a_codes [M][K], a_scales [M][K/128]       (from apex_quantize_act_int4_fp8)
+ *   w_codes [N][K], w_scales [N][K/group_w]   (apex_pack_weights_int4_fp8 or
+ *                                              apex_unpack_int4_fp8 + the packed scales)
+ * group_a == 128, group_w a multiple of 128 dividing K, K % 128 == 0, M, N >= 1 (ragged tiles
+ * handled).  a_codes / w_codes 16-byte aligned, scales and y 2-byte aligned.  No workspace:
+ * tiles of 128 tokens x 256 outputs are never split.  Codes that are not E4M3 values of
+ * integers in [-8, 7] give undefined results.
+ */
+apex_status_t apex_w4a4_gemm_fp8(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                 int32_t group_w, const void *a_codes, const void *a_scales,
+                                 const void *w_codes, const void *w_scales, void *y_f16,
+                                 void *stream);
+
+/*
+ * Parity export of the E4M3-carrier GEMM: every exact per-group partial, as
+ * apex_w4a4_group_partials, computed by the same tensor-core path as apex_w4a4_gemm_fp8
+ * (its fp32 partials stored as int32).
+ */
+apex_status_t apex_w4a4_group_partials_fp8(int64_t M, int64_t N, int64_t K,
+                                           const void *a_codes, const void *w_codes,
+                                           int32_t *partials_i32, void *stream);
 
 /*
  * Debug / parity export: the exact integer partial of every 128-wide K-group,
@@ -221,6 +287,15 @@ apex_status_t apex_debug_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t sms,
  * time limit.  -1 turns it off.  Used only to test the timeout path; never needed by callers.
  */
 void apex_debug_withhold_step(int32_t step);
+
+/*
+ * Test hook: the next apex_w4a4_group_partials call on this host thread (on != 0) divides
+ * the work as apex_w4a4_gemm does when given its workspace -- tiles split over several
+ * CTAs, in stream-K pieces -- instead of whole tiles.  Every (tile, K-group) is still
+ * handled by one CTA, which stores its partials, so the export needs no scratch; the hook
+ * checks the split plans' K ranges bit for bit.  It applies to one call, then resets.
+ */
+void apex_debug_partials_split(int32_t on);
 
 /*
  * Tracing hook: the next apex_w4a4_gemm launch on this host thread writes timestamps for

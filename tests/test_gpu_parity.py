@@ -139,6 +139,47 @@ def test_group_partials_quantized_workload(apex):
     assert np.array_equal(host(out).astype(np.int64), ref)
 
 
+def partials(apex, ap, wp, M, N, K, split):
+    out = torch.full((K // 128, M, N), -1, dtype=torch.int32, device="cuda")
+    apex.apex_debug_partials_split(split)
+    apex.apex_w4a4_group_partials(M, N, K, ap, wp, out)
+    torch.cuda.synchronize()
+    check_status(apex)
+    return host(out).astype(np.int64)
+
+
+@pytest.mark.parametrize("split", [False, True])
+def test_group_partials_full_decode_size(apex, split):
+    """Every per-group partial of the headline decode shape (16 x 8192 x 8192, all 64 K-groups,
+    every K coordinate and swizzle phase), bit-exact, on the GPU-quantized operands, whose
+    packing is itself checked against the oracle; with split=True the work is divided as the
+    bench's GEMM divides it (each tile over a 2-CTA cluster on a B200)."""
+    g = synth.workloads()["decode_m16_n8192_k8192"]
+    a, w = synth.make(g)
+    ap, _ = apex.quantize_act(dev(a), 128)
+    wp, _ = apex.pack_weights(dev(w), 128)
+    torch.cuda.synchronize()
+    ap_ref, _ = oracle.quantize_pack(a, 128)
+    wp_ref, _ = oracle.quantize_pack(w, 128)
+    assert np.array_equal(host(ap), ap_ref) and np.array_equal(host(wp), wp_ref)
+    ref = oracle.group_partials(ap_ref, wp_ref, g.M, g.N, g.K, 128, 128)
+    assert np.array_equal(partials(apex, ap, wp, g.M, g.N, g.K, split), ref)
+
+
+# Split plans on a 148-SM B200: 2-, 3- and 4-way cluster splits, a 9-way split through
+# global memory, true stream-K (CTAs holding pieces of two tiles) with 16-, 64- and
+# 128-token tiles, and ragged M and N.
+@pytest.mark.parametrize("M,N,K", [(16, 9472, 1024), (16, 6272, 1536), (5, 4736, 2048),
+                                   (16, 2048, 8192), (16, 12800, 1024), (64, 6400, 1024),
+                                   (200, 6400, 1024), (33, 1000, 2560)])
+def test_group_partials_split_plans_bit_exact(apex, M, N, K):
+    rng = np.random.default_rng(M + 3 * N + K)
+    ap = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)   # includes -8 nibbles
+    wp = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    ref = oracle.group_partials(ap, wp, M, N, K, 128, 128)
+    assert np.array_equal(partials(apex, dev(ap), dev(wp), M, N, K, True), ref)
+
+
 # ------------------------------------------------------------------ GEMM output
 
 
@@ -276,15 +317,15 @@ def test_gemm_large_workloads_sampled_rows(apex, name):
     cand |= set(rng.integers(0, g.M, size=min(g.M, 12)).tolist())
     rows = np.array(sorted(cand), dtype=np.int64)
     ap_h, sa_h, wp_h, sw_h = host(ap), host(sa), host(wp), host(sw)
-    # the GPU-packed operands are themselves checked against the oracle's quantizer
-    ap_ref, sa_ref = oracle.quantize_pack(a[rows], 128)
-    assert np.array_equal(ap_h[rows], ap_ref)
-    assert np.array_equal(sa_h[rows].view(np.uint16), sa_ref.view(np.uint16))
-    wrows = np.array(sorted({0, g.N - 1, 4097 % g.N, 77}), dtype=np.int64)
-    wp_ref, sw_ref = oracle.quantize_pack(w[wrows], g.gw)
-    assert np.array_equal(wp_h[wrows], wp_ref)
-    assert np.array_equal(sw_h[wrows].view(np.uint16), sw_ref.view(np.uint16))
-    ref = oracle.gemm(ap_h, sa_h, wp_h, sw_h, g.M, g.N, g.K, 128, g.gw, rows=rows)
+    # the GPU-packed operands are themselves checked against the oracle's quantizer, whole,
+    # before any of them serves as oracle input
+    ap_ref, sa_ref = oracle.quantize_pack(a, 128)
+    assert np.array_equal(ap_h, ap_ref)
+    assert np.array_equal(sa_h.view(np.uint16), sa_ref.view(np.uint16))
+    wp_ref, sw_ref = oracle.quantize_pack(w, g.gw)
+    assert np.array_equal(wp_h, wp_ref)
+    assert np.array_equal(sw_h.view(np.uint16), sw_ref.view(np.uint16))
+    ref = oracle.gemm(ap_ref, sa_ref, wp_ref, sw_ref, g.M, g.N, g.K, 128, g.gw, rows=rows)
     got = host(y)[rows].astype(np.float64)
     # max|ref| over the whole output is at least the sampled max: using the sampled max
     # makes the absolute term of the bound no looser than the stated rule.

@@ -1,10 +1,13 @@
-"""The allocation-free GEMM entry point, checked against the workspace-taking one.
+"""The allocation-free GEMM entry point, checked against the oracle and against the
+workspace-taking entry point.
 
 apex_w4a4_gemm_noalloc serves callers that cannot allocate device memory while they run
 (runtimes that budget every device byte in advance, plugin hosts whose allocator is off
 limits, latency-critical paths that must avoid cudaMalloc/cudaFree stalls).  Its split-K
 scratch is a fixed array inside the library, shared by every call on a device, so two
 calls in a row also check that the second one does not see the first one's leftovers.
+Both entry points take the same work plan and the same fixed-order split-K reduction, so
+their outputs must be bit-identical, not merely close.
 
 This file is collected last, so a run that stops at its first failure has already run
 every other test; it also passes when run alone in a fresh process.
@@ -28,18 +31,35 @@ def apex():
     return m
 
 
-@pytest.mark.parametrize("M,N,K,gw", [(16, 2048, 8192, 128), (32, 1024, 4096, 512),
-                                      (16, 256, 512, 128)])
-def test_noalloc_matches_workspace_gemm_twice(apex, M, N, K, gw):
-    a = synth.activations(M, K, "normal", 70 + M)
-    w = synth.weights(N, K, 70 + N)
-    a_d = torch.from_numpy(a).cuda()
-    w_d = torch.from_numpy(w).cuda()
-    ap, sa = apex.quantize_act(a_d, 128)
-    wp, sw = apex.pack_weights(w_d, gw)
+def operands(apex, M, N, K, gw, seed):
+    """GPU-quantized operands, checked bit for bit against the oracle's quantizer, and the
+    oracle's fp64 GEMM of them."""
+    a = synth.activations(M, K, "normal", seed + M)
+    w = synth.weights(N, K, seed + N)
+    ap, sa = apex.quantize_act(torch.from_numpy(a).cuda(), 128)
+    wp, sw = apex.pack_weights(torch.from_numpy(w).cuda(), gw)
+    torch.cuda.synchronize()
+    ap_ref, sa_ref = oracle.quantize_pack(a, 128)
+    wp_ref, sw_ref = oracle.quantize_pack(w, gw)
+    assert np.array_equal(ap.cpu().numpy(), ap_ref)
+    assert np.array_equal(wp.cpu().numpy(), wp_ref)
+    assert np.array_equal(sa.cpu().numpy().view(np.uint16), sa_ref.view(np.uint16))
+    assert np.array_equal(sw.cpu().numpy().view(np.uint16), sw_ref.view(np.uint16))
+    ref = oracle.gemm(ap_ref, sa_ref, wp_ref, sw_ref, M, N, K, 128, gw)
+    return (ap, sa, wp, sw), ref
+
+
+# (16, 16384, 8192): 128 tiles on 148 SMs, a true stream-K plan in which CTAs hold pieces of
+# two tiles and use the shared arrival counters for both; (16, 2048, 8192): every tile split
+# 9 ways through global memory; (32, 1024, 4096, 512): coarse weight groups; (16, 256, 512):
+# whole tiles, no scratch at all.
+@pytest.mark.parametrize("M,N,K,gw", [(16, 16384, 8192, 128), (16, 2048, 8192, 128),
+                                      (32, 1024, 4096, 512), (16, 256, 512, 128)])
+def test_noalloc_matches_oracle_and_workspace_gemm_twice(apex, M, N, K, gw):
+    (ap, sa, wp, sw), ref = operands(apex, M, N, K, gw, 70)
     ws = apex.workspace(M, N, K, 128, gw)
-    y_ref = torch.empty((M, N), dtype=torch.float16, device="cuda")
-    apex.apex_w4a4_gemm(M, N, K, 128, gw, ap, sa, wp, sw, y_ref, ws)
+    y_ws = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    apex.apex_w4a4_gemm(M, N, K, 128, gw, ap, sa, wp, sw, y_ws, ws)
     outs = []
     for _ in range(2):
         y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
@@ -47,11 +67,35 @@ def test_noalloc_matches_workspace_gemm_twice(apex, M, N, K, gw):
         outs.append(y)
     torch.cuda.synchronize()
     assert apex.apex_get_device_status() == 0
-    ref = y_ref.cpu().numpy().astype(np.float64)
+    ok, ratio = oracle.within_tolerance(y_ws.cpu().numpy().astype(np.float64), ref)
+    assert ok, f"apex_w4a4_gemm outside tolerance (worst err/bound {ratio:.3f})"
     for y in outs:
-        got = y.cpu().numpy().astype(np.float64)
-        ok, ratio = oracle.within_tolerance(got, ref)
-        assert ok, f"no-alloc output differs from apex_w4a4_gemm (worst err/bound {ratio:.3f})"
+        assert torch.equal(y.view(torch.int16), y_ws.view(torch.int16)), \
+            "no-alloc output is not bit-identical to apex_w4a4_gemm"
+        ok, ratio = oracle.within_tolerance(y.cpu().numpy().astype(np.float64), ref)
+        assert ok, f"no-alloc output outside tolerance (worst err/bound {ratio:.3f})"
+
+
+def test_noalloc_recovers_after_a_timed_out_call(apex):
+    # A call whose pipeline gives up (one bulk copy withheld, 50 ms wait limit) leaves its
+    # split-K counters wherever it stopped; the next call clears them and is exact again.
+    M, N, K = 16, 2048, 8192
+    (ap, sa, wp, sw), ref = operands(apex, M, N, K, 128, 80)
+    y = torch.zeros((M, N), dtype=torch.float16, device="cuda")
+    apex.apex_set_wait_limit_ns(50_000_000)
+    try:
+        apex.apex_debug_withhold_step(1)
+        apex.apex_w4a4_gemm_noalloc(M, N, K, 128, 128, ap, sa, wp, sw, y)
+        assert apex.apex_get_device_status() == apex.APEX_ERR_TIMEOUT
+    finally:
+        apex.apex_debug_withhold_step(-1)
+        apex.apex_set_wait_limit_ns(2_000_000_000)
+    y2 = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+    apex.apex_w4a4_gemm_noalloc(M, N, K, 128, 128, ap, sa, wp, sw, y2)
+    torch.cuda.synchronize()
+    assert apex.apex_get_device_status() == 0
+    ok, ratio = oracle.within_tolerance(y2.cpu().numpy().astype(np.float64), ref)
+    assert ok, f"call after the timeout outside tolerance (worst err/bound {ratio:.3f})"
 
 
 def test_noalloc_refuses_problems_beyond_its_scratch(apex):
