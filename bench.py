@@ -171,11 +171,16 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ the apex arm
 
-EXPANDED_MIN_M = 128   # from this many tokens on, the step uses the expanded activation form
+WIDE_MIN_M = 128   # from this many tokens on, the step uses one-byte operand forms
+FORM_OVERRIDE = None   # set by --form
 
 
 def activation_form(M: int) -> str:
-    return "expanded" if M >= EXPANDED_MIN_M else "packed"
+    """Operand form of the step: packed int4 (few tokens: memory-bound), or E4M3 codes of the
+    same int4 values for many tokens (compute-bound; the E4M3-carrier GEMM)."""
+    if FORM_OVERRIDE:
+        return FORM_OVERRIDE
+    return "fp8" if M >= WIDE_MIN_M else "packed"
 
 
 class Problem:
@@ -184,6 +189,7 @@ class Problem:
     def __init__(self, apex, torch, g: synth.Gemm, copies: int):
         self.form = activation_form(g.M)
         self.expanded = self.form == "expanded"
+        self.fp8 = self.form == "fp8"
         self.g = g
         a, w = synth.make(g)
         self.a_host = a
@@ -192,13 +198,14 @@ class Problem:
         self.wp, self.sw, self.ap, self.sa = [], [], [], []
         a_d = torch.from_numpy(a).to(dev)
         w_d = torch.from_numpy(w).to(dev)
-        wp0, sw0 = apex.pack_weights(w_d, g.gw)
+        # the weights are quantized once, offline, in the form the GEMM reads
+        wp0, sw0 = apex.pack_weights_fp8(w_d, g.gw) if self.fp8 else apex.pack_weights(w_d, g.gw)
         del w_d
         for c in range(copies):
             self.x.append(a_d if c == 0 else a_d.clone())
             self.wp.append(wp0 if c == 0 else wp0.clone())
             self.sw.append(sw0 if c == 0 else sw0.clone())
-            self.ap.append(torch.empty((g.M, g.K if self.expanded else g.K // 2),
+            self.ap.append(torch.empty((g.M, g.K // 2 if self.form == "packed" else g.K),
                                        dtype=torch.uint8, device=dev))
             self.sa.append(torch.empty((g.M, g.K // 128), dtype=torch.float16, device=dev))
         self.y = torch.empty((g.M, g.N), dtype=torch.float16, device=dev)
@@ -214,18 +221,28 @@ def copies_for(g: synth.Gemm, l2_bytes: int) -> int:
     return c
 
 
+def quantizer_of(apex, form):
+    return {"packed": apex.apex_quantize_act_int4,
+            "expanded": apex.apex_quantize_act_int4_expanded,
+            "fp8": apex.apex_quantize_act_int4_fp8}[form]
+
+
+def gemm_call(apex, form, g, a, sa, w, sw, y, ws, stream):
+    if form == "fp8":
+        apex.apex_w4a4_gemm_fp8(g.M, g.N, g.K, 128, g.gw, a, sa, w, sw, y, stream)
+    else:
+        gemm = apex.apex_w4a4_gemm_expanded if form == "expanded" else apex.apex_w4a4_gemm
+        gemm(g.M, g.N, g.K, 128, g.gw, a, sa, w, sw, y, ws, None, stream)
+
+
 def apex_quantize(apex, p: Problem, i: int, stream):
     g, c = p.g, i % p.copies
-    if p.expanded:
-        apex.apex_quantize_act_int4_expanded(p.x[c], g.M, g.K, 128, p.ap[c], p.sa[c], stream)
-    else:
-        apex.apex_quantize_act_int4(p.x[c], g.M, g.K, 128, p.ap[c], p.sa[c], stream)
+    quantizer_of(apex, p.form)(p.x[c], g.M, g.K, 128, p.ap[c], p.sa[c], stream)
 
 
 def apex_gemm(apex, p: Problem, i: int, stream):
     g, c = p.g, i % p.copies
-    gemm = apex.apex_w4a4_gemm_expanded if p.expanded else apex.apex_w4a4_gemm
-    gemm(g.M, g.N, g.K, 128, g.gw, p.ap[c], p.sa[c], p.wp[c], p.sw[c], p.y, p.ws, None, stream)
+    gemm_call(apex, p.form, g, p.ap[c], p.sa[c], p.wp[c], p.sw[c], p.y, p.ws, stream)
 
 
 def apex_step(apex, p: Problem, i: int, stream):
@@ -318,8 +335,7 @@ def e2e_workload(apex, torch, g, steps, warmup, p: Problem):
     ev = lambda: torch.cuda.Event()
     in_ready, q_done = [ev() for _ in range(C)], [ev() for _ in range(C)]
     y_ready, out_done = [ev() for _ in range(2)], [ev() for _ in range(2)]
-    gemm = apex.apex_w4a4_gemm_expanded if p.expanded else apex.apex_w4a4_gemm
-    quant = apex.apex_quantize_act_int4_expanded if p.expanded else apex.apex_quantize_act_int4
+    quant = quantizer_of(apex, p.form)
 
     def step(j, first):
         c, b = j % C, j % 2
@@ -333,8 +349,7 @@ def e2e_workload(apex, torch, g, steps, warmup, p: Problem):
             stream.wait_event(out_done[b])             # that output's previous copy is done
         quant(p.x[c], g.M, g.K, 128, p.ap[c], p.sa[c], stream)
         q_done[c].record(stream)
-        gemm(g.M, g.N, g.K, 128, g.gw, p.ap[c], p.sa[c], p.wp[c], p.sw[c], y_dev[b], p.ws,
-             None, stream)
+        gemm_call(apex, p.form, g, p.ap[c], p.sa[c], p.wp[c], p.sw[c], y_dev[b], p.ws, stream)
         y_ready[b].record(stream)
         with torch.cuda.stream(copy_out):
             copy_out.wait_event(y_ready[b])
@@ -716,7 +731,11 @@ def main():
     ap.add_argument("--no-second", action="store_true", help="skip the M=4096 companion line")
     ap.add_argument("--sweep", action="store_true",
                     help="instead of the headline line, one line per sweep / MLP workload")
+    ap.add_argument("--form", choices=["packed", "expanded", "fp8"], default=None,
+                    help="operand form of every step (default: by the number of tokens)")
     args = ap.parse_args()
+    global FORM_OVERRIDE
+    FORM_OVERRIDE = args.form
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank, world, local = dist_init(args.gpus)

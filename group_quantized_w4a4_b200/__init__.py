@@ -24,6 +24,9 @@ __all__ = [
     "apex_w4a4_gemm_noalloc", "apex_quantize_act_int4_expanded", "apex_w4a4_gemm_expanded",
     "apex_w4a4_gemm_quant", "apex_w4a4_gemm_expanded_quant",
     "quantize_act_expanded",
+    "apex_quantize_act_int4_fp8", "apex_pack_weights_int4_fp8", "apex_unpack_int4_fp8",
+    "apex_w4a4_gemm_fp8", "apex_w4a4_group_partials_fp8", "quantize_act_fp8",
+    "pack_weights_fp8", "gemm_fp8",
     "apex_w4a4_gemm_workspace_size", "apex_w4a4_group_partials", "apex_get_device_status",
     "apex_set_wait_limit_ns", "apex_status_string", "apex_debug_withhold_step",
     "apex_debug_trace_next_gemm", "apex_debug_gemm_plan", "apex_debug_partials_split",
@@ -82,6 +85,16 @@ def load_library(build_if_missing: bool = True):
             fn = getattr(lib, name)
             fn.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P, P, I32, P, SZ, P]
             fn.restype = st
+        lib.apex_quantize_act_int4_fp8.argtypes = [P, I64, I64, I32, P, P, P]
+        lib.apex_quantize_act_int4_fp8.restype = st
+        lib.apex_pack_weights_int4_fp8.argtypes = [P, I64, I64, I32, P, P, P]
+        lib.apex_pack_weights_int4_fp8.restype = st
+        lib.apex_unpack_int4_fp8.argtypes = [P, I64, I64, P, P]
+        lib.apex_unpack_int4_fp8.restype = st
+        lib.apex_w4a4_gemm_fp8.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P]
+        lib.apex_w4a4_gemm_fp8.restype = st
+        lib.apex_w4a4_group_partials_fp8.argtypes = [I64, I64, I64, P, P, P, P]
+        lib.apex_w4a4_group_partials_fp8.restype = st
         lib.apex_w4a4_gemm_noalloc.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P]
         lib.apex_w4a4_gemm_noalloc.restype = st
         lib.apex_w4a4_gemm_workspace_size.argtypes = [I64, I64, I64, I32, I32]
@@ -222,6 +235,71 @@ def quantize_act_expanded(x, group_a: int = 128, stream=None):
     scales = torch.empty((M, K // group_a), dtype=torch.float16, device=x.device)
     apex_quantize_act_int4_expanded(x, M, K, group_a, q8, scales, stream)
     return q8, scales
+
+
+def apex_quantize_act_int4_fp8(x_f16, M, K, group_a, x_codes, x_scales_f16, stream=None):
+    _check(load_library().apex_quantize_act_int4_fp8(_ptr(x_f16), M, K, group_a, _ptr(x_codes),
+                                                     _ptr(x_scales_f16), _stream(stream)),
+           "apex_quantize_act_int4_fp8")
+
+
+def apex_pack_weights_int4_fp8(w_f16, N, K, group_w, w_codes, w_scales_f16, stream=None):
+    _check(load_library().apex_pack_weights_int4_fp8(_ptr(w_f16), N, K, group_w, _ptr(w_codes),
+                                                     _ptr(w_scales_f16), _stream(stream)),
+           "apex_pack_weights_int4_fp8")
+
+
+def apex_unpack_int4_fp8(packed, rows, K, codes, stream=None):
+    _check(load_library().apex_unpack_int4_fp8(_ptr(packed), rows, K, _ptr(codes),
+                                               _stream(stream)),
+           "apex_unpack_int4_fp8")
+
+
+def apex_w4a4_gemm_fp8(M, N, K, group_a, group_w, a_codes, a_scales, w_codes, w_scales, y_f16,
+                       stream=None):
+    _check(load_library().apex_w4a4_gemm_fp8(M, N, K, group_a, group_w, _ptr(a_codes),
+                                             _ptr(a_scales), _ptr(w_codes), _ptr(w_scales),
+                                             _ptr(y_f16), _stream(stream)),
+           "apex_w4a4_gemm_fp8")
+
+
+def apex_w4a4_group_partials_fp8(M, N, K, a_codes, w_codes, partials_i32, stream=None):
+    _check(load_library().apex_w4a4_group_partials_fp8(M, N, K, _ptr(a_codes), _ptr(w_codes),
+                                                       _ptr(partials_i32), _stream(stream)),
+           "apex_w4a4_group_partials_fp8")
+
+
+def quantize_act_fp8(x, group_a: int = 128, stream=None):
+    """fp16 [M, K] CUDA tensor -> (E4M3 codes uint8 [M, K], scales fp16 [M, K/group_a])."""
+    import torch
+    M, K = x.shape
+    codes = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((M, K // group_a), dtype=torch.float16, device=x.device)
+    apex_quantize_act_int4_fp8(x, M, K, group_a, codes, scales, stream)
+    return codes, scales
+
+
+def pack_weights_fp8(w, group_w: int = 128, stream=None):
+    """fp16 [N, K] CUDA tensor -> (E4M3 codes uint8 [N, K], scales fp16 [N, K/group_w])."""
+    import torch
+    N, K = w.shape
+    codes = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((N, K // group_w), dtype=torch.float16, device=w.device)
+    apex_pack_weights_int4_fp8(w, N, K, group_w, codes, scales, stream)
+    return codes, scales
+
+
+def gemm_fp8(a_codes, a_scales, w_codes, w_scales, group_a=128, group_w=128, out=None,
+             stream=None):
+    """Y = W4A4 GEMM of E4M3-coded operands -> fp16 [M, N]."""
+    import torch
+    M, K = a_codes.shape
+    N = w_codes.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=a_codes.device)
+    apex_w4a4_gemm_fp8(M, N, K, group_a, group_w, a_codes, a_scales, w_codes, w_scales, out,
+                       stream)
+    return out
 
 
 def apex_w4a4_gemm_noalloc(M, N, K, group_a, group_w, a_packed, a_scales, w_packed, w_scales,

@@ -447,11 +447,15 @@ F8Plan make_f8_plan(int64_t M, int64_t N, int sms_override = 0) {
   return p;
 }
 
-template <bool DUMP>
+#ifndef APEX_F8_EPI_WARPS
+#define APEX_F8_EPI_WARPS 8
+#endif
+
+template <int MODE>
 apex_status_t launch_f8(const F8Plan& p, const CUtensorMap& ma, const CUtensorMap& mb,
                         const apex::F8Args& a, cudaStream_t s) {
-  using C = apex::F8Cfg<DUMP>;
-  auto kern = apex::w4a4_gemm_f8_kernel<DUMP>;
+  using C = apex::F8Cfg<APEX_F8_EPI_WARPS>;
+  auto kern = apex::w4a4_gemm_f8_kernel<MODE, APEX_F8_EPI_WARPS>;
   static thread_local int attr_dev = -1;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return APEX_ERR_CUDA;
@@ -543,8 +547,11 @@ apex_status_t apex_w4a4_gemm_fp8(int64_t M, int64_t N, int64_t K, int32_t group_
   a.sw = static_cast<const __half*>(w_scales);
   a.y = static_cast<__half*>(y_f16);
   a.sa_vec = a.G % 8 == 0 && aligned(a_scales, 16);
+  a.sw_vec = group_w == 128 && a.G % 8 == 0 && aligned(w_scales, 16);
   a.y_vec = N % 8 == 0 && aligned(y_f16, 16);
-  return launch_f8<false>(p, ma, mb, a, static_cast<cudaStream_t>(stream));
+  // per-channel weight groups: the weight scale factors out of the K sum
+  return group_w == K ? launch_f8<apex::F8_PER_CHANNEL>(p, ma, mb, a, static_cast<cudaStream_t>(stream))
+                      : launch_f8<apex::F8_GROUPED>(p, ma, mb, a, static_cast<cudaStream_t>(stream));
 }
 
 apex_status_t apex_w4a4_group_partials_fp8(int64_t M, int64_t N, int64_t K, const void* a_codes,
@@ -560,7 +567,7 @@ apex_status_t apex_w4a4_group_partials_fp8(int64_t M, int64_t N, int64_t K, cons
   st = f8_setup(M, N, K, 128, a_codes, w_codes, p, a, ma, mb);
   if (st != APEX_OK) return st;
   a.dump = partials_i32;
-  return launch_f8<true>(p, ma, mb, a, static_cast<cudaStream_t>(stream));
+  return launch_f8<apex::F8_DUMP>(p, ma, mb, a, static_cast<cudaStream_t>(stream));
 }
 
 apex_status_t apex_pack_weights_int4(const void* w_f16, int64_t N, int64_t K, int32_t group_w,

@@ -45,6 +45,11 @@
 
 namespace apex {
 
+// Epilogue modes: per-group weight scales (any weight group), one weight scale per row for
+// the whole K (per-channel weight groups: the scale is applied once, after the sum), or the
+// partials export.
+enum F8Mode : int { F8_GROUPED = 0, F8_PER_CHANNEL = 1, F8_DUMP = 2 };
+
 struct F8Args {
   int M, N, K;
   int G;             // K / 128
@@ -62,7 +67,9 @@ struct F8Args {
   unsigned long long wait_ns;
 };
 
-template <bool DUMP>
+// EW: epilogue warps, 8 (128 columns a thread, 32-column partial loads double-buffered) or
+// 16 (64 columns a thread, twice the warps to cover latencies, 16-column loads).
+template <int EW>
 struct F8Cfg {
   static constexpr int BM = 128;                   // tokens per tile
   static constexpr int BN = 256;                   // weight rows per tile
@@ -72,16 +79,22 @@ struct F8Cfg {
   static constexpr int STAGE = A_BYTES + B_BYTES;  // 48 KB
   static constexpr int SLOTS = 2;                  // partial slots of BN columns
   static constexpr int TMEM_COLS = SLOTS * BN;     // 512
-  static constexpr int EPI_WARPS = 8;
-  static constexpr int EPI_THREADS = EPI_WARPS * 32;
-  static constexpr int THREADS = 128 + EPI_THREADS;  // 384
-  static constexpr int REGS_LAUNCH = 168;          // 3 warps x 32 x 168 <= 16384 per quarter
-  static constexpr int REGS_CTRL = 40;
-  static constexpr int REGS_EPI = 232;
+  static constexpr int EPI_WARPS = EW;
+  static constexpr int EPI_THREADS = EW * 32;
+  static constexpr int THREADS = 128 + EPI_THREADS;
+  // registers: what __launch_bounds__(THREADS, 1) allows (warps per SM sub-partition x 32 x
+  // registers <= 16384), then the first warpgroup keeps REGS_CTRL and the epilogue takes
+  // REGS_EPI
+  static constexpr int REGS_LAUNCH = EW == 8 ? 168 : 96;
+  static constexpr int REGS_CTRL = EW == 8 ? 40 : 24;
+  static constexpr int REGS_EPI = EW == 8 ? 232 : 112;
   static_assert(128 * REGS_CTRL + EPI_THREADS * REGS_EPI <= THREADS * REGS_LAUNCH,
                 "register budgets fit the block's pool");
-  static constexpr int CPT = BN / 2;               // columns per epilogue thread (128)
-  static constexpr int SWB = 8 * BN * 4;           // one staged block of weight scales (fp32)
+  static constexpr int CPT = BN * 4 / EW;          // columns per epilogue thread
+  static constexpr int LC = EW == 8 ? 32 : 16;     // columns per tensor-memory load
+  static constexpr bool DBUF = EW == 8;            // next load in flight during the current
+  static constexpr int SPT = 8 * BN / EPI_THREADS;  // staged weight scales per thread
+  static constexpr int SWB = 8 * BN * 2;           // one staged block of weight scales (fp16)
   static constexpr int OFF_STAGE = 0;
   static constexpr int OFF_SW = NS * STAGE;
   static constexpr int OFF_BAR = OFF_SW + 2 * SWB;
@@ -91,6 +104,7 @@ struct F8Cfg {
   static_assert(STAGE % 1024 == 0 && A_BYTES % 1024 == 0, "swizzle atoms stay aligned");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(TMEM_COLS <= 512, "tensor memory budget");
+  static_assert(CPT % LC == 0 && (SPT == 8 || SPT == 4), "epilogue split");
 };
 
 // Tile t -> (token tile, weight tile): bands of 8 token tiles, weight tiles across each band,
@@ -106,20 +120,45 @@ __device__ __forceinline__ void f8_tile(const F8Args& a, int t, int& tm, int& tn
   tn = r / rows;
 }
 
-// The 8 fp16 scales of groups gb8 .. gb8+7 of one row (raw bits, zeros outside [0, G) and
-// for rows outside the matrix): one 16-byte load when `vec` (8 consecutive scale groups,
-// 16-byte aligned), else one load per group; gpg = K-groups per scale group.
-__device__ __forceinline__ uint4 scale_block8(const __half* base, int row, int rows, int ld,
-                                              int gb8, int G, int gpg, bool vec) {
+// The NG (8 or 4) fp16 scales of groups g0 .. g0+NG-1 of one row (raw bits, packed two per
+// 32-bit word; zeros outside [0, G) and for rows outside the matrix): one 16- or 8-byte load
+// when `vec` (consecutive scale groups, aligned), else one load per group; gpg = K-groups per
+// scale group.
+template <int NG>
+__device__ __forceinline__ uint4 scale_block(const __half* base, int row, int rows, int ld,
+                                             int g0, int G, int gpg, bool vec) {
   if (row >= rows) return make_uint4(0, 0, 0, 0);
   const __half* r = base + (size_t)row * ld;
-  if (vec) return __ldg(reinterpret_cast<const uint4*>(r + gb8));
-  uint32_t h[8];
+  if (vec) {
+    if constexpr (NG == 8) return __ldg(reinterpret_cast<const uint4*>(r + g0));
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(r + g0));
+    return make_uint4(v.x, v.y, 0u, 0u);
+  }
+  uint32_t h[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    h[j] = gb8 + j < G ? (uint32_t)__half_as_ushort(r[(gb8 + j) / gpg]) : 0u;
+  for (int j = 0; j < NG; ++j)
+    h[j] = g0 + j < G ? (uint32_t)__half_as_ushort(r[(g0 + j) / gpg]) : 0u;
   return make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
                     h[6] | (h[7] << 16));
+}
+
+__device__ __forceinline__ uint16_t half_bits_at(const uint4& v, int j) {
+  const uint32_t w = j < 2 ? v.x : j < 4 ? v.y : j < 6 ? v.z : v.w;
+  return (uint16_t)((j & 1) ? (w >> 16) : (w & 0xFFFFu));
+}
+
+// (sa * sw_lo, sa * sw_hi) in fp32 from fp16 bits: one mixed-precision fma each (f16 inputs,
+// f32 result, + 0), exact, since the product of two fp16 values fits fp32's significand and
+// range.
+__device__ __forceinline__ float2 scale_pair(uint32_t sw2, uint16_t sa) {
+  float lo, hi;
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "fma.rn.f32.f16 %0, %3, l, 0f00000000;\n\t"
+      "fma.rn.f32.f16 %1, %3, h, 0f00000000;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(sw2), "h"(sa));
+  return make_float2(lo, hi);
 }
 
 __device__ __forceinline__ float half_at(const uint4& v, int j) {
@@ -133,16 +172,18 @@ __device__ __forceinline__ uint32_t half2_bits(float2 v) {
 }
 
 
-template <bool DUMP>
-__global__ void __launch_bounds__(F8Cfg<DUMP>::THREADS, 1)
-    __maxnreg__(F8Cfg<DUMP>::REGS_LAUNCH) w4a4_gemm_f8_kernel(const __grid_constant__ CUtensorMap tmA,
+template <int MODE, int EW>
+__global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
+    w4a4_gemm_f8_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const F8Args args) {
-  using C = F8Cfg<DUMP>;
+  using C = F8Cfg<EW>;
+  constexpr bool DUMP = MODE == F8_DUMP;
+  constexpr bool PERCH = MODE == F8_PER_CHANNEL;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* stages = smem + C::OFF_STAGE;
-  float* s_sw = reinterpret_cast<float*>(smem + C::OFF_SW);
+  uint16_t* s_sw = reinterpret_cast<uint16_t*>(smem + C::OFF_SW);   // fp16 bits
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* full = bars;                 // stage loaded (TMA bytes)
   uint64_t* empty = full + C::NS;        // stage read by its MMAs (commit)
@@ -189,11 +230,10 @@ __global__ void __launch_bounds__(F8Cfg<DUMP>::THREADS, 1)
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(s_tmem);
   volatile int* abort_flag = s_abort;
   volatile int* never = s_never;
-  if (warp < 4)
+  // Role dispatch by warpgroup first, so that each register budget covers exactly the code
+  // of its warpgroup.
+  if (warp < 4) {
     regs_dec<C::REGS_CTRL>();
-  else
-    regs_inc<C::REGS_EPI>();
-
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     grid_dep_wait();
@@ -253,13 +293,15 @@ __global__ void __launch_bounds__(F8Cfg<DUMP>::THREADS, 1)
     __syncwarp();
     mbar_wait(smem_u32(mma_done), 0u, lim, never);
     __syncwarp();
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_inc<C::REGS_EPI>();
     // ------------------------------------------------------------ epilogue
     grid_dep_wait();   // scales and outputs are global memory
-    const int ew = warp - 4;                    // 0..7
-    const int et = threadIdx.x - 128;           // 0..255: the weight column it stages
+    const int ew = warp - 4;                    // 0 .. EW-1
+    const int et = threadIdx.x - 128;           // stages weight column et % 256
     const int lq = warp & 3;                    // tensor-memory lane quarter of this warp
-    const int ch = ew >> 2;                     // column half: columns 128*ch .. +127
+    const int ch = ew >> 2;                     // columns CPT*ch .. +CPT-1
     const int row = 32 * lq + lane;             // token of the tile
     const uint32_t t_lane = (uint32_t)(32 * lq) << 16;
     constexpr uint32_t EB = 1;                  // named barrier of the epilogue warps
@@ -269,10 +311,19 @@ __global__ void __launch_bounds__(F8Cfg<DUMP>::THREADS, 1)
     int it = 0;
     int b = 0;   // flat 8-group block counter: its weight scales are staged in s_sw[b & 1]
 
-    // weight scales of one block: thread et stages column et, all 8 groups
-    auto stage_sw = [&](float* blk, const uint4& v) {
+    // weight scales of one block, as fp16 bits: thread et stages column et % 256, groups
+    // SPT*(et / 256) .. +SPT-1
+    const int sw_col = et & 255, sw_g0 = C::SPT * (et >> 8);
+    auto stage_sw = [&](uint16_t* blk, const uint4& v) {
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int j = 0; j < 8; ++j) blk[j * C::BN + et] = half_at(v, j);
+      for (int j = 0; j < C::SPT; ++j)
+        blk[(sw_g0 + j) * C::BN + sw_col] =
+            (uint16_t)((j & 1) ? (w[j / 2] >> 16) : (w[j / 2] & 0xFFFFu));
+    };
+    auto load_sw = [&](int tn, int gb8) {
+      return scale_block<C::SPT>(args.sw, tn * C::BN + sw_col, args.N, args.Gw, gb8 + sw_g0, G,
+                                 args.gpg, sw_vec);
     };
     // the first block's scales before the first group
     int t = blockIdx.x;
@@ -280,9 +331,9 @@ __global__ void __launch_bounds__(F8Cfg<DUMP>::THREADS, 1)
     if (t < args.T && !DUMP) {
       int tm, tn;
       f8_tile(args, t, tm, tn);
-      stage_sw(s_sw, scale_block8(args.sw, tn * C::BN + et, args.N, args.Gw, 0, G, args.gpg,
-                                  sw_vec));
-      sa_c = scale_block8(args.sa, tm * C::BM + row, args.M, G, 0, G, 1, sa_vec);
+      if constexpr (!PERCH)
+        stage_sw(s_sw, load_sw(tn, 0));
+      sa_c = scale_block<8>(args.sa, tm * C::BM + row, args.M, G, 0, G, 1, sa_vec);
     }
     aborted = bar_red_or(EB, C::EPI_THREADS, false);
     for (; !aborted && t < args.T; t += args.P) {
@@ -302,11 +353,10 @@ __global__ void __launch_bounds__(F8Cfg<DUMP>::THREADS, 1)
         const int ngb = more ? gb8 + 8 : 0;
         uint4 sw_n = make_uint4(0, 0, 0, 0), sa_n = make_uint4(0, 0, 0, 0);
         if (have_next) {
-          sw_n = scale_block8(args.sw, ntn * C::BN + et, args.N, args.Gw, ngb, G, args.gpg,
-                              sw_vec);
-          sa_n = scale_block8(args.sa, ntm * C::BM + row, args.M, G, ngb, G, 1, sa_vec);
+          if constexpr (!PERCH) sw_n = load_sw(ntn, ngb);
+          sa_n = scale_block<8>(args.sa, ntm * C::BM + row, args.M, G, ngb, G, 1, sa_vec);
         }
-        const float* swb = s_sw + (b & 1) * (C::SWB / 4) + ch * C::CPT;
+        const uint16_t* swb = s_sw + (b & 1) * (C::SWB / 2) + ch * C::CPT;
         const int je = min(8, G - gb8);
         for (int j = 0; j < je && ok; ++j, ++it) {
           const int sl = it % C::SLOTS;
@@ -315,54 +365,104 @@ __global__ void __launch_bounds__(F8Cfg<DUMP>::THREADS, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t td = tbase + t_lane + sl * C::BN + ch * C::CPT;
-          const float saf = half_at(sa_c, j);
+          const uint16_t sa_h = half_bits_at(sa_c, j);
+          const float saf = __half2float(__ushort_as_half(sa_h));
           const float2 sa2 = make_float2(saf, saf);
-          const float* swj = swb + j * C::BN;
-          // four 32-column loads, the next one in flight while the current one is used
-          uint32_t p[2][32];
-          tmem_ld32_nowait(td, p[0]);
-          tmem_ld_wait32(p[0]);
+          const uint16_t* swj = swb + j * C::BN;
+          // NCH loads of LC columns; with DBUF the next one is in flight while the current
+          // one is used
+          constexpr int NCH = C::CPT / C::LC;
+          uint32_t p[C::DBUF ? 2 : 1][C::LC];
+          auto ld = [&](int cc, uint32_t* dst) {
+            if constexpr (C::LC == 32) tmem_ld32_nowait(td + 32 * cc, dst);
+            else tmem_ld16_nowait(td + 16 * cc, dst);
+          };
+          auto ld_wait = [&](uint32_t* dst) {
+            if constexpr (C::LC == 32) tmem_ld_wait32(dst);
+            else tmem_ld_wait16(dst);
+          };
+          auto release = [&]() {   // every load of the slot has completed
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&tempty[sl]));
+          };
+          if constexpr (C::DBUF) {
+            ld(0, p[0]);
+            ld_wait(p[0]);
+          }
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t* pc = p[cc & 1];
-            if (cc < 3) tmem_ld32_nowait(td + 32 * (cc + 1), p[(cc + 1) & 1]);
-            if constexpr (DUMP) {
-              int32_t* dst = args.dump + ((size_t)(gb8 + j) * args.M + m) * args.N + n0 + cc * 32;
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (m < args.M && n0 + cc * 32 + e < args.N)
-                  dst[e] = __float2int_rn(__uint_as_float(pc[e]));
+          for (int cc = 0; cc < NCH; ++cc) {
+            uint32_t* pc = p[C::DBUF ? (cc & 1) : 0];
+            if constexpr (C::DBUF) {
+              if (cc + 1 < NCH) ld(cc + 1, p[(cc + 1) & 1]);
             } else {
+              ld(cc, pc);
+              ld_wait(pc);
+              if (cc == NCH - 1) release();
+            }
+            if constexpr (DUMP) {
+              int32_t* dst =
+                  args.dump + ((size_t)(gb8 + j) * args.M + m) * args.N + n0 + cc * C::LC;
 #pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const float4 s4 = *reinterpret_cast<const float4*>(swj + cc * 32 + 4 * q);
-                const float2 s_a = __fmul2_rn(make_float2(s4.x, s4.y), sa2);
-                const float2 s_b = __fmul2_rn(make_float2(s4.z, s4.w), sa2);
-                acc[cc * 16 + 2 * q] = __ffma2_rn(
-                    make_float2(__uint_as_float(pc[4 * q]), __uint_as_float(pc[4 * q + 1])),
-                    s_a, acc[cc * 16 + 2 * q]);
-                acc[cc * 16 + 2 * q + 1] = __ffma2_rn(
-                    make_float2(__uint_as_float(pc[4 * q + 2]), __uint_as_float(pc[4 * q + 3])),
-                    s_b, acc[cc * 16 + 2 * q + 1]);
+              for (int e = 0; e < C::LC; ++e)
+                if (m < args.M && n0 + cc * C::LC + e < args.N)
+                  dst[e] = __float2int_rn(__uint_as_float(pc[e]));
+            } else if constexpr (PERCH) {
+              // one weight scale for all of K: acc += P * sa here, times sw after the sum
+#pragma unroll
+              for (int q = 0; q < C::LC / 2; ++q)
+                acc[cc * (C::LC / 2) + q] = __ffma2_rn(
+                    make_float2(__uint_as_float(pc[2 * q]), __uint_as_float(pc[2 * q + 1])), sa2,
+                    acc[cc * (C::LC / 2) + q]);
+            } else {
+              // s = sa * sw, exact in fp32, from the fp16 scales in one mixed-precision fma
+#pragma unroll
+              for (int q = 0; q < C::LC / 8; ++q) {
+                const uint4 w8 = *reinterpret_cast<const uint4*>(swj + cc * C::LC + 8 * q);
+                const uint32_t w[4] = {w8.x, w8.y, w8.z, w8.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  const int e = cc * (C::LC / 2) + 4 * q + h;
+                  acc[e] = __ffma2_rn(make_float2(__uint_as_float(pc[8 * q + 2 * h]),
+                                                  __uint_as_float(pc[8 * q + 2 * h + 1])),
+                                      scale_pair(w[h], sa_h), acc[e]);
+                }
               }
             }
-            if (cc < 3) tmem_ld_wait32(p[(cc + 1) & 1]);
-            if (cc == 2) {
-              // every load of the slot has completed: hand it back to the MMA
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(smem_u32(&tempty[sl]));
+            if constexpr (C::DBUF) {
+              if (cc + 1 < NCH) ld_wait(p[(cc + 1) & 1]);
+              if (cc == NCH - 2) release();
             }
           }
         }
         // the next block's weight scales into the other buffer; one barrier per block (also
         // the epilogue's one decision to give up, so no warp is left waiting here)
-        if (have_next) stage_sw(s_sw + ((b + 1) & 1) * (C::SWB / 4), sw_n);
+        if constexpr (!PERCH) {
+          if (have_next) stage_sw(s_sw + ((b + 1) & 1) * (C::SWB / 2), sw_n);
+        }
         aborted = bar_red_or(EB, C::EPI_THREADS, !ok);
         if (aborted) break;
         sa_c = sa_n;
       }
       if (aborted) break;
+      if constexpr (PERCH) {
+        // the row's one weight scale, applied to the finished sum
+        // (8 columns at a time: the compiler barrier keeps the loads from all being hoisted
+        // next to the 128 accumulators)
+        const __half* swc = args.sw + (size_t)n0 * args.Gw;
+#pragma unroll
+        for (int e0 = 0; e0 < C::CPT / 2; e0 += 4) {
+          float sv[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            sv[c] = n0 + 2 * e0 + c < args.N ? __half2float(swc[(size_t)(2 * e0 + c) * args.Gw])
+                                            : 0.0f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            acc[e0 + e] = __fmul2_rn(acc[e0 + e], make_float2(sv[2 * e], sv[2 * e + 1]));
+          asm volatile("" ::: "memory");
+        }
+      }
       if constexpr (!DUMP) {
         // the finished tile: this thread's token row, 128 consecutive outputs
         if (m < args.M) {

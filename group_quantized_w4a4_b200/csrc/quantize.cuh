@@ -68,9 +68,13 @@ __device__ __forceinline__ int quant1(float f, const QScale& qs) {
 }
 
 // Two integer-valued floats (|v| <= 8) as E4M3 codes, exact: lo in bits 0..7, hi in 8..15.
+// A zero is always coded +0 (0x00): q = 0 reached from a negative value is -0.0 in fp32,
+// and adding +0 turns it into +0 (IEEE round to nearest).
 __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+      : "=h"(r)
+      : "f"(__fadd_rn(hi, 0.0f)), "f"(__fadd_rn(lo, 0.0f)));
   return r;
 }
 

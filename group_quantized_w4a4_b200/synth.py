@@ -80,18 +80,20 @@ class Gemm:
         return 2.0 * self.M * self.N * self.K
 
     def gemm_bytes(self, form: str = "packed") -> int:
-        """Algorithmic HBM bytes of one GEMM call: A, packed W, fp16 scales, fp16 Y.  A is
-        packed int4 plus scales ("packed") or one byte per element plus scales
-        ("expanded")."""
+        """Algorithmic HBM bytes of one GEMM call: A, W, fp16 scales, fp16 Y.  A is packed
+        int4 plus scales ("packed") or one byte per element plus scales ("expanded");
+        "fp8" has one byte per element for both A and W (E4M3 codes of the int4 values)."""
         M, N, K = self.M, self.N, self.K
         a = {"packed": M * K // 2 + 2 * M * (K // self.ga),
-             "expanded": M * K + 2 * M * (K // self.ga)}[form]
-        return a + N * K // 2 + 2 * N * (K // self.gw) + 2 * M * N
+             "expanded": M * K + 2 * M * (K // self.ga),
+             "fp8": M * K + 2 * M * (K // self.ga)}[form]
+        w = N * K if form == "fp8" else N * K // 2     # fp8: one byte per weight
+        return a + w + 2 * N * (K // self.gw) + 2 * M * N
 
     def quant_bytes(self, form: str = "packed") -> int:
         """Algorithmic HBM bytes of the online activation quantizer."""
         M, K = self.M, self.K
-        return 2 * M * K + (M * K if form == "expanded" else M * K // 2) + 2 * M * (K // self.ga)
+        return 2 * M * K + (M * K // 2 if form == "packed" else M * K) + 2 * M * (K // self.ga)
 
 
 def workloads() -> dict:
