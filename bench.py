@@ -623,7 +623,66 @@ def run_sweep(args, rank, world, local):
     for m in (2048, 16):
         line = chain_line(apex, torch, m, steps, args.warmup, world)
         lines.append(line)
+    lines.append(dual_line(apex, torch, synth.workloads()[SECOND_WORKLOAD], steps, args.warmup,
+                           world, l2, peaks, peaks_kind, int8_peak))
     return lines if rank == 0 else None
+
+
+def dual_line(apex, torch, g, steps, warmup, world, l2, peaks, peaks_kind, int8_peak):
+    """The outlier dual path on a workload with persistent outlier channels (the prefill
+    workload: 1% of K, x20, the same for every token): the step is the dual quantizer (the
+    outlier channels to fp16, the rest to E4M3 codes) and the dual GEMM (the 4-bit groups plus
+    the 16-bit outlier K-steps), timed as the plain step is."""
+    dev = torch.device("cuda")
+    a, w = synth.make(g)
+    ch = synth.outlier_channels(g.K, g.seed * 16 + 2)
+    C = len(ch)
+    Cp = -(-C // 64) * 64
+    ch_d = torch.from_numpy(ch.astype(np.int32)).to(dev)
+    w_d = torch.from_numpy(w).to(dev)
+    w_out = torch.empty((g.N, Cp), dtype=torch.float16, device=dev)
+    apex.apex_gather_weight_columns(w_d, g.N, g.K, ch_d, C, w_out, Cp)
+    wc, sw = apex.pack_weights_fp8(w_d, g.gw)
+    del w_d
+    copies = copies_for(g, l2)
+    xs = [torch.from_numpy(a).to(dev) for _ in range(copies)]
+    qs = [torch.empty((g.M, g.K), dtype=torch.uint8, device=dev) for _ in range(copies)]
+    ss = [torch.empty((g.M, g.K // 128), dtype=torch.float16, device=dev) for _ in range(copies)]
+    xo = [torch.empty((g.M, Cp), dtype=torch.float16, device=dev) for _ in range(copies)]
+    y = torch.empty((g.M, g.N), dtype=torch.float16, device=dev)
+
+    def quant(i, s):
+        c = i % copies
+        apex.apex_quantize_act_int4_dual(xs[c], g.M, g.K, 128, ch_d, C, apex.APEX_FORM_FP8,
+                                         qs[c], ss[c], xo[c], Cp, s)
+
+    def gemm(i, s):
+        c = i % copies
+        apex.apex_w4a4_gemm_fp8_dual(g.M, g.N, g.K, 128, g.gw, qs[c], ss[c], wc, sw, xo[c],
+                                     w_out, Cp, y, s)
+
+    def step(i, s):
+        quant(i, s)
+        gemm(i, s)
+
+    stream = torch.cuda.current_stream()
+    for i in range(max(warmup, copies)):
+        step(i, stream)
+    torch.cuda.synchronize()
+    if apex.apex_get_device_status() != 0:
+        raise RuntimeError("device status not clean after the dual-path warm-up")
+    tot, _ = timed_graph(torch, step, steps, warmup, world)
+    gm, _ = timed_graph(torch, gemm, steps, warmup, world)
+    qm, _ = timed_graph(torch, quant, steps, warmup, world)
+    ms, gm, qm = (max_over_ranks(v / steps, world) for v in (tot, gm, qm))
+    return {"sweep": f"{g.name}_outlier_dual", "M": g.M, "N": g.N, "K": g.K,
+            "outlier_channels": C, "Cp": Cp, "steps": steps, "activation_form": "fp8",
+            "step_ms": round(ms, 5), "gemm_ms": round(gm, 5), "quantize_ms": round(qm, 5),
+            "step_TOPS": round(job_throughput(g.ops, ms, world), 2),
+            "roofline": roofline_obj(g, gm, peaks, peaks_kind, int8_peak=int8_peak,
+                                     form="fp8"),
+            "what": ("outlier channels in fp16 through extra kind::f16 K-steps of the same "
+                     "GEMM, the rest W4A4-g128; ops counted as the plain GEMM's 2*M*N*K")}
 
 
 def chain_line(apex, torch, M, steps, warmup, world):

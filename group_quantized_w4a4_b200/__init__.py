@@ -27,6 +27,7 @@ __all__ = [
     "apex_quantize_act_int4_fp8", "apex_pack_weights_int4_fp8", "apex_unpack_int4_fp8",
     "apex_w4a4_gemm_fp8", "apex_w4a4_group_partials_fp8", "quantize_act_fp8",
     "pack_weights_fp8", "gemm_fp8",
+    "apex_gather_weight_columns", "apex_quantize_act_int4_dual", "apex_w4a4_gemm_fp8_dual",
     "apex_w4a4_gemm_workspace_size", "apex_w4a4_group_partials", "apex_get_device_status",
     "apex_set_wait_limit_ns", "apex_status_string", "apex_debug_withhold_step",
     "apex_debug_trace_next_gemm", "apex_debug_gemm_plan", "apex_debug_partials_split",
@@ -39,6 +40,10 @@ APEX_ERR_UNSUPPORTED = 2
 APEX_ERR_ALIGNMENT = 3
 APEX_ERR_CUDA = 4
 APEX_ERR_TIMEOUT = 5
+
+APEX_FORM_PACKED = 0     # output forms of apex_quantize_act_int4_dual
+APEX_FORM_EXPANDED = 1
+APEX_FORM_FP8 = 2
 
 _lock = threading.Lock()
 _lib = None
@@ -95,6 +100,14 @@ def load_library(build_if_missing: bool = True):
         lib.apex_w4a4_gemm_fp8.restype = st
         lib.apex_w4a4_group_partials_fp8.argtypes = [I64, I64, I64, P, P, P, P]
         lib.apex_w4a4_group_partials_fp8.restype = st
+        lib.apex_gather_weight_columns.argtypes = [P, I64, I64, P, I32, P, I32, P]
+        lib.apex_gather_weight_columns.restype = st
+        lib.apex_quantize_act_int4_dual.argtypes = [P, I64, I64, I32, P, I32, I32, P, P, P,
+                                                    I32, P]
+        lib.apex_quantize_act_int4_dual.restype = st
+        lib.apex_w4a4_gemm_fp8_dual.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P, I32,
+                                                P, P]
+        lib.apex_w4a4_gemm_fp8_dual.restype = st
         lib.apex_w4a4_gemm_noalloc.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P]
         lib.apex_w4a4_gemm_noalloc.restype = st
         lib.apex_w4a4_gemm_workspace_size.argtypes = [I64, I64, I64, I32, I32]
@@ -300,6 +313,31 @@ def gemm_fp8(a_codes, a_scales, w_codes, w_scales, group_a=128, group_w=128, out
     apex_w4a4_gemm_fp8(M, N, K, group_a, group_w, a_codes, a_scales, w_codes, w_scales, out,
                        stream)
     return out
+
+
+def apex_gather_weight_columns(w_f16, N, K, channels_i32, C, w_out_f16, Cp, stream=None):
+    _check(load_library().apex_gather_weight_columns(_ptr(w_f16), N, K, _ptr(channels_i32), C,
+                                                     _ptr(w_out_f16), Cp, _stream(stream)),
+           "apex_gather_weight_columns")
+
+
+def apex_quantize_act_int4_dual(x_f16, M, K, group_a, channels_i32, C, form, x_q, x_scales_f16,
+                                x_out_f16, Cp, stream=None):
+    _check(load_library().apex_quantize_act_int4_dual(_ptr(x_f16), M, K, group_a,
+                                                      _ptr(channels_i32), C, int(form),
+                                                      _ptr(x_q), _ptr(x_scales_f16),
+                                                      _ptr(x_out_f16), Cp, _stream(stream)),
+           "apex_quantize_act_int4_dual")
+
+
+def apex_w4a4_gemm_fp8_dual(M, N, K, group_a, group_w, a_codes, a_scales, w_codes, w_scales,
+                            x_out_f16, w_out_f16, Cp, y_f16, stream=None):
+    _check(load_library().apex_w4a4_gemm_fp8_dual(M, N, K, group_a, group_w, _ptr(a_codes),
+                                                  _ptr(a_scales), _ptr(w_codes),
+                                                  _ptr(w_scales), _ptr(x_out_f16),
+                                                  _ptr(w_out_f16), Cp, _ptr(y_f16),
+                                                  _stream(stream)),
+           "apex_w4a4_gemm_fp8_dual")
 
 
 def apex_w4a4_gemm_noalloc(M, N, K, group_a, group_w, a_packed, a_scales, w_packed, w_scales,

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "apex_w4a4.h"
+#include "dual.cuh"
 #include "gemm.cuh"
 #include "gemm_f8.cuh"
 #include "ptx.cuh"
@@ -105,6 +106,21 @@ bool make_expanded_map(CUtensorMap* map, const void* base, int64_t rows, int64_t
   cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1u, 1u};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 2-D map over fp16 [rows][cols] (the outlier dual path's compact operands); box = 64
+// halves (128 bytes) x box_rows rows, 128-byte swizzle, zeros outside.
+bool make_f16_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -451,11 +467,12 @@ F8Plan make_f8_plan(int64_t M, int64_t N, int sms_override = 0) {
 #define APEX_F8_EPI_WARPS 8
 #endif
 
-template <int MODE>
+template <int MODE, bool DUAL = false>
 apex_status_t launch_f8(const F8Plan& p, const CUtensorMap& ma, const CUtensorMap& mb,
-                        const apex::F8Args& a, cudaStream_t s) {
+                        const apex::F8Args& a, cudaStream_t s, const CUtensorMap& mxo_,
+                        const CUtensorMap& mwo_) {
   using C = apex::F8Cfg<APEX_F8_EPI_WARPS>;
-  auto kern = apex::w4a4_gemm_f8_kernel<MODE, APEX_F8_EPI_WARPS>;
+  auto kern = apex::w4a4_gemm_f8_kernel<MODE, APEX_F8_EPI_WARPS, DUAL>;
   static thread_local int attr_dev = -1;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return APEX_ERR_CUDA;
@@ -465,7 +482,11 @@ apex_status_t launch_f8(const F8Plan& p, const CUtensorMap& ma, const CUtensorMa
       return APEX_ERR_CUDA;
     attr_dev = dev;
   }
-  return cuda_status(launch_pdl(kern, (unsigned)p.P, C::THREADS, (size_t)C::SMEM, s, ma, mb, a));
+  // without the outlier dual path the outlier maps are never read: the operand maps stand in
+  const CUtensorMap& mxo = a.NO > 0 ? mxo_ : ma;
+  const CUtensorMap& mwo = a.NO > 0 ? mwo_ : mb;
+  return cuda_status(
+      launch_pdl(kern, (unsigned)p.P, C::THREADS, (size_t)C::SMEM, s, ma, mb, mxo, mwo, a));
 }
 
 // The shared part of apex_w4a4_gemm_fp8 and the partials export: checks, plan, maps.
@@ -550,8 +571,9 @@ apex_status_t apex_w4a4_gemm_fp8(int64_t M, int64_t N, int64_t K, int32_t group_
   a.sw_vec = group_w == 128 && a.G % 8 == 0 && aligned(w_scales, 16);
   a.y_vec = N % 8 == 0 && aligned(y_f16, 16);
   // per-channel weight groups: the weight scale factors out of the K sum
-  return group_w == K ? launch_f8<apex::F8_PER_CHANNEL>(p, ma, mb, a, static_cast<cudaStream_t>(stream))
-                      : launch_f8<apex::F8_GROUPED>(p, ma, mb, a, static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return group_w == K ? launch_f8<apex::F8_PER_CHANNEL>(p, ma, mb, a, s, ma, mb)
+                      : launch_f8<apex::F8_GROUPED>(p, ma, mb, a, s, ma, mb);
 }
 
 apex_status_t apex_w4a4_group_partials_fp8(int64_t M, int64_t N, int64_t K, const void* a_codes,
@@ -567,7 +589,7 @@ apex_status_t apex_w4a4_group_partials_fp8(int64_t M, int64_t N, int64_t K, cons
   st = f8_setup(M, N, K, 128, a_codes, w_codes, p, a, ma, mb);
   if (st != APEX_OK) return st;
   a.dump = partials_i32;
-  return launch_f8<apex::F8_DUMP>(p, ma, mb, a, static_cast<cudaStream_t>(stream));
+  return launch_f8<apex::F8_DUMP>(p, ma, mb, a, static_cast<cudaStream_t>(stream), ma, mb);
 }
 
 apex_status_t apex_pack_weights_int4(const void* w_f16, int64_t N, int64_t K, int32_t group_w,
@@ -811,6 +833,113 @@ const char* apex_status_string(apex_status_t status) {
     case APEX_ERR_TIMEOUT: return "device pipeline wait timed out";
   }
   return "unknown status";
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- outlier dual path
+
+namespace {
+
+apex_status_t check_outlier_args(int64_t K, const void* channels, int32_t C, int32_t Cp) {
+  if (!channels || C < 1 || C > K || Cp < C || Cp % 64) return APEX_ERR_INVALID_ARG;
+  if (!aligned(channels, 4)) return APEX_ERR_ALIGNMENT;
+  return APEX_OK;
+}
+
+unsigned grid_for(int64_t work, int threads, int per_sm) {
+  int64_t blocks = (work + threads - 1) / threads;
+  const int64_t cap = (int64_t)dev_info().sms * per_sm;
+  if (blocks > cap) blocks = cap;
+  return (unsigned)(blocks < 1 ? 1 : blocks);
+}
+
+}  // namespace
+
+extern "C" {
+
+apex_status_t apex_gather_weight_columns(const void* w_f16, int64_t N, int64_t K,
+                                         const void* channels, int32_t C, void* w_out_f16,
+                                         int32_t Cp, void* stream) {
+  if (!w_f16 || !w_out_f16 || N <= 0 || K <= 0) return APEX_ERR_INVALID_ARG;
+  apex_status_t st = check_outlier_args(K, channels, C, Cp);
+  if (st != APEX_OK) return st;
+  if (!aligned(w_f16, 2) || !aligned(w_out_f16, 16)) return APEX_ERR_ALIGNMENT;
+  cudaError_t e = launch_pdl(apex::gather_columns_kernel, grid_for(N * (int64_t)Cp, 256, 16), 256,
+                             0, static_cast<cudaStream_t>(stream),
+                             static_cast<const __half*>(w_f16), N, K,
+                             static_cast<const int32_t*>(channels), (int)C,
+                             static_cast<__half*>(w_out_f16), (int)Cp);
+  if (e != cudaSuccess) return APEX_ERR_CUDA;
+  return cuda_status(cudaPeekAtLastError());
+}
+
+apex_status_t apex_quantize_act_int4_dual(const void* x_f16, int64_t M, int64_t K,
+                                          int32_t group_a, const void* channels, int32_t C,
+                                          int32_t form, void* x_q, void* x_scales_f16,
+                                          void* x_out_f16, int32_t Cp, void* stream) {
+  if (!x_f16 || !x_q || !x_scales_f16 || !x_out_f16) return APEX_ERR_INVALID_ARG;
+  if (M <= 0 || K <= 0 || K % 128) return APEX_ERR_INVALID_ARG;
+  if (form < APEX_FORM_PACKED || form > APEX_FORM_FP8) return APEX_ERR_INVALID_ARG;
+  if (group_a != 128) return APEX_ERR_UNSUPPORTED;
+  apex_status_t st = check_outlier_args(K, channels, C, Cp);
+  if (st != APEX_OK) return st;
+  if (!aligned(x_f16, 16) || !aligned(x_q, form == APEX_FORM_PACKED ? 4 : 8) ||
+      !aligned(x_scales_f16, 2) || !aligned(x_out_f16, 16))
+    return APEX_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned nb = grid_for(((M * (K / 128) + 1) / 2) * 32, 128, 32);
+  const __half* xh = static_cast<const __half*>(x_f16);
+  const int32_t* ch = static_cast<const int32_t*>(channels);
+  uint8_t* q = static_cast<uint8_t*>(x_q);
+  __half* sc = static_cast<__half*>(x_scales_f16);
+  __half* xo = static_cast<__half*>(x_out_f16);
+  cudaError_t e;
+  if (form == APEX_FORM_FP8)
+    e = launch_pdl(apex::quantize_dual_kernel<apex::FORM_E4M3>, nb, 128, 0, s, xh, M, K, ch,
+                   (int)C, q, sc, xo, (int)Cp);
+  else if (form == APEX_FORM_EXPANDED)
+    e = launch_pdl(apex::quantize_dual_kernel<apex::FORM_EXPANDED>, nb, 128, 0, s, xh, M, K, ch,
+                   (int)C, q, sc, xo, (int)Cp);
+  else
+    e = launch_pdl(apex::quantize_dual_kernel<apex::FORM_PACKED>, nb, 128, 0, s, xh, M, K, ch,
+                   (int)C, q, sc, xo, (int)Cp);
+  if (e != cudaSuccess) return APEX_ERR_CUDA;
+  return cuda_status(cudaPeekAtLastError());
+}
+
+apex_status_t apex_w4a4_gemm_fp8_dual(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                      int32_t group_w, const void* a_codes,
+                                      const void* a_scales, const void* w_codes,
+                                      const void* w_scales, const void* x_out_f16,
+                                      const void* w_out_f16, int32_t Cp, void* y_f16,
+                                      void* stream) {
+  apex_status_t st = check_gemm_args(M, N, K, group_a, group_w);
+  if (st != APEX_OK) return st;
+  if (!a_scales || !w_scales || !y_f16 || !x_out_f16 || !w_out_f16) return APEX_ERR_INVALID_ARG;
+  if (Cp < 64 || Cp % 64 || Cp > K) return APEX_ERR_INVALID_ARG;
+  if (!aligned(a_scales, 2) || !aligned(w_scales, 2) || !aligned(y_f16, 2) ||
+      !aligned(x_out_f16, 16) || !aligned(w_out_f16, 16))
+    return APEX_ERR_ALIGNMENT;
+  F8Plan p;
+  apex::F8Args a;
+  CUtensorMap ma, mb, mxo, mwo;
+  st = f8_setup(M, N, K, group_w, a_codes, w_codes, p, a, ma, mb);
+  if (st != APEX_OK) return st;
+  memset(&mxo, 0, sizeof(mxo));
+  memset(&mwo, 0, sizeof(mwo));
+  if (!make_f16_map(&mxo, x_out_f16, M, Cp, 128) || !make_f16_map(&mwo, w_out_f16, N, Cp, 256))
+    return APEX_ERR_CUDA;
+  a.sa = static_cast<const __half*>(a_scales);
+  a.sw = static_cast<const __half*>(w_scales);
+  a.y = static_cast<__half*>(y_f16);
+  a.sa_vec = a.G % 8 == 0 && aligned(a_scales, 16);
+  a.sw_vec = group_w == 128 && a.G % 8 == 0 && aligned(w_scales, 16);
+  a.y_vec = N % 8 == 0 && aligned(y_f16, 16);
+  a.NO = Cp / 64;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return group_w == K ? launch_f8<apex::F8_PER_CHANNEL, true>(p, ma, mb, a, s, mxo, mwo)
+                      : launch_f8<apex::F8_GROUPED, true>(p, ma, mb, a, s, mxo, mwo);
 }
 
 }  // extern "C"

@@ -65,6 +65,10 @@ struct F8Args {
   __half* y;         // [M][N]
   int32_t* dump;     // [G][M][N] per-group partials (export kernel only)
   unsigned long long wait_ns;
+  // The outlier dual path (0: none): NO extra K-steps of 64 fp16 channels per tile, from the
+  // maps tmXo (x_out [M][64*NO]) and tmWo (w_out [N][64*NO]), multiplied by kind::f16 MMAs
+  // and added with unit scale after the 4-bit groups.
+  int NO;
 };
 
 // EW: epilogue warps, 8 (128 columns a thread, 32-column partial loads double-buffered) or
@@ -172,10 +176,13 @@ __device__ __forceinline__ uint32_t half2_bits(float2 v) {
 }
 
 
-template <int MODE, int EW>
+// DUAL: the outlier dual path's K-steps are compiled in (args.NO of them; else none).
+template <int MODE, int EW, bool DUAL = false>
 __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
     w4a4_gemm_f8_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const F8Args args) {
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmXo,
+                        const __grid_constant__ CUtensorMap tmWo, const F8Args args) {
   using C = F8Cfg<EW>;
   constexpr bool DUMP = MODE == F8_DUMP;
   constexpr bool PERCH = MODE == F8_PER_CHANNEL;
@@ -198,6 +205,8 @@ __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
   const int lane = threadIdx.x & 31;
   const uint64_t lim = args.wait_ns;
   const int G = args.G;
+  const int NO = DUAL ? args.NO : 0;
+  const int GT = args.G + NO;        // K-steps per tile: the 4-bit groups, then the outliers
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NS; ++i) {
@@ -216,6 +225,10 @@ __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (NO > 0) {
+      tma_prefetch_desc(&tmXo);
+      tma_prefetch_desc(&tmWo);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(s_tmem), C::TMEM_COLS);
@@ -242,7 +255,7 @@ __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
     for (int t = blockIdx.x; ok && t < args.T; t += args.P) {
       int tm, tn;
       f8_tile(args, t, tm, tn);
-      for (int g = 0; g < G; ++g, ++it) {
+      for (int g = 0; g < GT; ++g, ++it) {
         const int st = it % C::NS;
         ok = mbar_wait(smem_u32(&empty[st]), ((uint32_t)(it / C::NS) & 1u) ^ 1u, lim, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
@@ -251,8 +264,13 @@ __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
           const uint32_t fb = smem_u32(&full[st]);
           uint8_t* sa_dst = stages + st * C::STAGE;
           mbar_arrive_expect_tx(fb, C::STAGE);
-          tma_load_2d(smem_u32(sa_dst), &tmA, fb, g * 128, tm * C::BM);
-          tma_load_2d(smem_u32(sa_dst + C::A_BYTES), &tmB, fb, g * 128, tn * C::BN);
+          if (g < G) {   // 128 E4M3 codes of each row: one K-group
+            tma_load_2d(smem_u32(sa_dst), &tmA, fb, g * 128, tm * C::BM);
+            tma_load_2d(smem_u32(sa_dst + C::A_BYTES), &tmB, fb, g * 128, tn * C::BN);
+          } else {       // 64 fp16 outlier channels of each row (the same 128 bytes a row)
+            tma_load_2d(smem_u32(sa_dst), &tmXo, fb, (g - G) * 64, tm * C::BM);
+            tma_load_2d(smem_u32(sa_dst + C::A_BYTES), &tmWo, fb, (g - G) * 64, tn * C::BN);
+          }
         }
         __syncwarp();
         last = it;
@@ -268,7 +286,7 @@ __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
     int it = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < args.T; t += args.P) {
-      for (int g = 0; g < G; ++g, ++it) {
+      for (int g = 0; g < GT; ++g, ++it) {
         const int st = it % C::NS, sl = it % C::SLOTS;
         ok = mbar_wait2(smem_u32(&full[st]), (uint32_t)(it / C::NS) & 1u,
                         smem_u32(&tempty[sl]), ((uint32_t)(it / C::SLOTS) & 1u) ^ 1u, lim,
@@ -280,9 +298,18 @@ __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
           const uint64_t a0 = smem_desc_k_sw128(smem_u32(stages + st * C::STAGE));
           const uint64_t b0 = smem_desc_k_sw128(smem_u32(stages + st * C::STAGE + C::A_BYTES));
           const uint32_t d = tbase + sl * C::BN;
+          // 32 bytes of K per MMA (+2 in 16-byte descriptor units): 32 E4M3 codes, or 16 fp16
+          // outlier channels (kind::f16; the descriptor's type fields read the same)
+          if (g < G) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j)   // K = 32 bytes per MMA: +2 in 16-byte descriptor units
-            umma_f8_ss(d, a0 + (uint64_t)(2 * j), b0 + (uint64_t)(2 * j), idesc, j > 0 ? 1u : 0u);
+            for (int j = 0; j < 4; ++j)
+              umma_f8_ss(d, a0 + (uint64_t)(2 * j), b0 + (uint64_t)(2 * j), idesc, j > 0 ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              umma_f16_ss(d, a0 + (uint64_t)(2 * j), b0 + (uint64_t)(2 * j), idesc,
+                          j > 0 ? 1u : 0u);
+          }
           umma_commit(smem_u32(&empty[st]));
           umma_commit(smem_u32(&tfull[sl]));
         }
@@ -314,16 +341,27 @@ __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
     // weight scales of one block, as fp16 bits: thread et stages column et % 256, groups
     // SPT*(et / 256) .. +SPT-1
     const int sw_col = et & 255, sw_g0 = C::SPT * (et >> 8);
+    // (per-channel weight groups: only the column's one scale, in group row 0)
     auto stage_sw = [&](uint16_t* blk, const uint4& v) {
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      if constexpr (PERCH) {
+        if (sw_g0 == 0) blk[sw_col] = (uint16_t)(v.x & 0xFFFFu);
+      } else {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int j = 0; j < C::SPT; ++j)
-        blk[(sw_g0 + j) * C::BN + sw_col] =
-            (uint16_t)((j & 1) ? (w[j / 2] >> 16) : (w[j / 2] & 0xFFFFu));
+        for (int j = 0; j < C::SPT; ++j)
+          blk[(sw_g0 + j) * C::BN + sw_col] =
+              (uint16_t)((j & 1) ? (w[j / 2] >> 16) : (w[j / 2] & 0xFFFFu));
+      }
     };
     auto load_sw = [&](int tn, int gb8) {
-      return scale_block<C::SPT>(args.sw, tn * C::BN + sw_col, args.N, args.Gw, gb8 + sw_g0, G,
-                                 args.gpg, sw_vec);
+      if constexpr (PERCH) {
+        const int n = tn * C::BN + sw_col;
+        return make_uint4(sw_g0 == 0 && n < args.N ? __half_as_ushort(args.sw[n]) : 0u, 0u, 0u,
+                          0u);
+      } else {
+        return scale_block<C::SPT>(args.sw, tn * C::BN + sw_col, args.N, args.Gw, gb8 + sw_g0,
+                                   G, args.gpg, sw_vec);
+      }
     };
     // the first block's scales before the first group
     int t = blockIdx.x;
@@ -331,8 +369,7 @@ __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
     if (t < args.T && !DUMP) {
       int tm, tn;
       f8_tile(args, t, tm, tn);
-      if constexpr (!PERCH)
-        stage_sw(s_sw, load_sw(tn, 0));
+      stage_sw(s_sw, load_sw(tn, 0));
       sa_c = scale_block<8>(args.sa, tm * C::BM + row, args.M, G, 0, G, 1, sa_vec);
     }
     aborted = bar_red_or(EB, C::EPI_THREADS, false);
@@ -353,7 +390,7 @@ __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
         const int ngb = more ? gb8 + 8 : 0;
         uint4 sw_n = make_uint4(0, 0, 0, 0), sa_n = make_uint4(0, 0, 0, 0);
         if (have_next) {
-          if constexpr (!PERCH) sw_n = load_sw(ntn, ngb);
+          sw_n = load_sw(ntn, ngb);
           sa_n = scale_block<8>(args.sa, ntm * C::BM + row, args.M, G, ngb, G, 1, sa_vec);
         }
         const uint16_t* swb = s_sw + (b & 1) * (C::SWB / 2) + ch * C::CPT;
@@ -437,35 +474,62 @@ __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
         }
         // the next block's weight scales into the other buffer; one barrier per block (also
         // the epilogue's one decision to give up, so no warp is left waiting here)
-        if constexpr (!PERCH) {
-          if (have_next) stage_sw(s_sw + ((b + 1) & 1) * (C::SWB / 2), sw_n);
-        }
+        if (have_next) stage_sw(s_sw + ((b + 1) & 1) * (C::SWB / 2), sw_n);
         aborted = bar_red_or(EB, C::EPI_THREADS, !ok);
         if (aborted) break;
         sa_c = sa_n;
       }
       if (aborted) break;
       if constexpr (PERCH) {
-        // the row's one weight scale, applied to the finished sum
-        // (8 columns at a time: the compiler barrier keeps the loads from all being hoisted
-        // next to the 128 accumulators)
-        const __half* swc = args.sw + (size_t)n0 * args.Gw;
+        // the row's one weight scale, applied to the finished sum of the 4-bit groups: it was
+        // staged with the tile's last block (every group row of the block holds it)
+        const uint16_t* swl = s_sw + ((b - 1) & 1) * (C::SWB / 2) + ch * C::CPT;
 #pragma unroll
-        for (int e0 = 0; e0 < C::CPT / 2; e0 += 4) {
-          float sv[8];
+        for (int e8 = 0; e8 < C::CPT; e8 += 8) {
+          const uint4 w8 = *reinterpret_cast<const uint4*>(swl + e8);
+          const uint32_t w[4] = {w8.x, w8.y, w8.z, w8.w};
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            sv[c] = n0 + 2 * e0 + c < args.N ? __half2float(swc[(size_t)(2 * e0 + c) * args.Gw])
-                                            : 0.0f;
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            acc[e0 + e] = __fmul2_rn(acc[e0 + e], make_float2(sv[2 * e], sv[2 * e + 1]));
-          asm volatile("" ::: "memory");
+          for (int h = 0; h < 4; ++h)
+            acc[e8 / 2 + h] = __fmul2_rn(acc[e8 / 2 + h],
+                                         make_float2(__half2float(__ushort_as_half((uint16_t)(w[h] & 0xFFFFu))),
+                                                     __half2float(__ushort_as_half((uint16_t)(w[h] >> 16)))));
         }
       }
       if constexpr (!DUMP) {
-        // the finished tile: this thread's token row, 128 consecutive outputs
-        if (m < args.M) {
+        // the outlier channels' 16-bit products, added with unit scale; a wait that gives up
+        // leaves the rest to the next block barrier (no warp can be left behind there)
+        for (int o = 0; o < NO && ok; ++o, ++it) {
+          const int sl = it % C::SLOTS;
+          ok = mbar_wait(smem_u32(&tfull[sl]), (uint32_t)(it / C::SLOTS) & 1u, lim, abort_flag);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t td = tbase + t_lane + sl * C::BN + ch * C::CPT;
+#pragma unroll
+          for (int cc = 0; cc < C::CPT / C::LC; ++cc) {
+            uint32_t p[C::LC];
+            if constexpr (C::LC == 32) {
+              tmem_ld32_nowait(td + 32 * cc, p);
+              tmem_ld_wait32(p);
+            } else {
+              tmem_ld16_nowait(td + 16 * cc, p);
+              tmem_ld_wait16(p);
+            }
+            if (cc == C::CPT / C::LC - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(smem_u32(&tempty[sl]));
+            }
+#pragma unroll
+            for (int q = 0; q < C::LC / 2; ++q)   // P * 1 + acc: one rounding, as an add
+              acc[cc * (C::LC / 2) + q] = __ffma2_rn(
+                  make_float2(__uint_as_float(p[2 * q]), __uint_as_float(p[2 * q + 1])),
+                  make_float2(1.0f, 1.0f), acc[cc * (C::LC / 2) + q]);
+          }
+        }
+        // the finished tile: this thread's token row, 128 consecutive outputs (after a wait
+        // that gave up, nothing: the next block barrier takes the decision to stop)
+        if (ok && m < args.M) {
           __half* dst = args.y + (size_t)m * args.N + n0;
           if (args.y_vec && n0 + C::CPT <= args.N) {
 #pragma unroll

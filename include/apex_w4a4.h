@@ -319,6 +319,59 @@ void apex_debug_partials_split(int32_t on);
  */
 void apex_debug_trace_next_gemm(uint64_t *trace, int32_t ctas, int32_t steps);
 
+/*
+ * ---- The outlier dual path ("OSC: Hardware Efficient W4A4 Quantization via Outlier
+ * Separation in Channel Dimension", abstract): a fixed set of input channels, the same for
+ * every token and chosen offline, bypasses 4-bit quantization and is multiplied in 16 bits;
+ * the rest goes through the W4A4 GEMM.  Here the 16-bit product runs inside the E4M3-carrier
+ * GEMM, as extra K-steps of every tile on the tensor cores (fp16 x fp16, fp32 accumulation),
+ * and is added to the fp32 result before the single fp16 rounding of Y.
+ *
+ * channels: device int32 [C], the outlier channel indices, sorted ascending, distinct, each
+ *   in [0, K) (a list that breaks this gives wrong values, never an out-of-bounds access).
+ *   1 <= C <= K.  Cp >= C, Cp % 64 == 0: the width of the compact fp16 operands, whose
+ *   columns C..Cp-1 are written as zeros.  channels 4-byte aligned.
+ */
+
+/* Output forms of apex_quantize_act_int4_dual. */
+#define APEX_FORM_PACKED 0   /* packed int4, as apex_quantize_act_int4 */
+#define APEX_FORM_EXPANDED 1 /* 16*q bytes, as apex_quantize_act_int4_expanded */
+#define APEX_FORM_FP8 2      /* E4M3 codes, as apex_quantize_act_int4_fp8 */
+
+/*
+ * Offline: the weights' outlier columns, w_out [N][Cp] fp16 (column c = w[:, channels[c]]),
+ * from w_f16 [N][K].  The 4-bit weights are quantized as usual (their outlier columns meet
+ * zero activations).  w_f16 2-byte, w_out_f16 16-byte aligned.
+ */
+apex_status_t apex_gather_weight_columns(const void *w_f16, int64_t N, int64_t K,
+                                         const void *channels, int32_t C, void *w_out_f16,
+                                         int32_t Cp, void *stream);
+
+/*
+ * Online: the activation quantizer (group_a must be 128) in the given form, with the
+ * outlier channels copied to x_out [M][Cp] fp16 (channel order of the list) and treated as
+ * zeros by the 4-bit path, so that they do not set its group scales.  x_f16 and x_out_f16
+ * 16-byte aligned; x_q 4-byte (packed) or 8-byte aligned; x_scales_f16 [M][K/128].
+ */
+apex_status_t apex_quantize_act_int4_dual(const void *x_f16, int64_t M, int64_t K,
+                                          int32_t group_a, const void *channels, int32_t C,
+                                          int32_t form, void *x_q, void *x_scales_f16,
+                                          void *x_out_f16, int32_t Cp, void *stream);
+
+/*
+ * The dual-path GEMM: Y = W4A4(a_codes, a_scales, w_codes, w_scales) + x_out . w_out^T, the
+ * 16-bit product accumulated in fp32 and added before the single fp16 rounding.  The operand
+ * rules of apex_w4a4_gemm_fp8; x_out_f16 [M][Cp] (from apex_quantize_act_int4_dual with
+ * APEX_FORM_FP8) and w_out_f16 [N][Cp] (apex_gather_weight_columns), both 16-byte aligned;
+ * 64 <= Cp <= K, Cp % 64 == 0.
+ */
+apex_status_t apex_w4a4_gemm_fp8_dual(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                      int32_t group_w, const void *a_codes,
+                                      const void *a_scales, const void *w_codes,
+                                      const void *w_scales, const void *x_out_f16,
+                                      const void *w_out_f16, int32_t Cp, void *y_f16,
+                                      void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -242,3 +242,114 @@ def test_gemm_fp8_argument_errors(apex):
     with pytest.raises(apex.ApexError) as e:
         apex.apex_w4a4_gemm_fp8(16, 128, 256, 128, 128, t[1:], h, t, h, h)   # misaligned
     assert e.value.code == apex.APEX_ERR_ALIGNMENT
+
+
+# ------------------------------------------------------------------ outlier dual path
+
+
+def dual_inputs(apex, x, w, ch, Cp, gw=128):
+    """Device operands of the dual path: the outlier list, the gathered weight columns, the
+    weight codes, and the dual quantizer's outputs (E4M3 codes, scales, x_out)."""
+    M, K = x.shape
+    N = w.shape[0]
+    ch_d = dev(np.ascontiguousarray(ch, dtype=np.int32))
+    w_d = dev(w)
+    w_out = torch.full((N, Cp), float("nan"), dtype=torch.float16, device="cuda")
+    apex.apex_gather_weight_columns(w_d, N, K, ch_d, len(ch), w_out, Cp)
+    wc, sw = apex.pack_weights_fp8(w_d, gw)
+    q = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    s = torch.empty((M, K // 128), dtype=torch.float16, device="cuda")
+    x_out = torch.full((M, Cp), float("nan"), dtype=torch.float16, device="cuda")
+    apex.apex_quantize_act_int4_dual(dev(x), M, K, 128, ch_d, len(ch), apex.APEX_FORM_FP8, q, s,
+                                     x_out, Cp)
+    return q, s, x_out, wc, sw, w_out
+
+
+@pytest.mark.parametrize("M,K,C,Cp", [(16, 1024, 11, 64), (37, 2048, 21, 64), (3, 256, 1, 64),
+                                      (130, 4096, 82, 128)])
+@pytest.mark.parametrize("form", [0, 1, 2])
+def test_quantize_dual_is_the_oracle_split_then_quantizer(apex, M, K, C, Cp, form):
+    x = synth.activations(M, K, "outlier", 70 + M)
+    ch = np.sort(np.random.default_rng(K + C).choice(K, size=C, replace=False))
+    ch_d = dev(ch.astype(np.int32))
+    q = torch.empty((M, K // 2 if form == 0 else K), dtype=torch.uint8, device="cuda")
+    s = torch.empty((M, K // 128), dtype=torch.float16, device="cuda")
+    x_out = torch.full((M, Cp), float("nan"), dtype=torch.float16, device="cuda")
+    apex.apex_quantize_act_int4_dual(dev(x), M, K, 128, ch_d, C, form, q, s, x_out, Cp)
+    torch.cuda.synchronize()
+    x_in, x_out_ref = oracle.split_outlier_channels(x, ch)
+    ap_ref, sa_ref = oracle.quantize_pack(x_in, 128)
+    qv = oracle.unpack(ap_ref, K).astype(np.int64)
+    if form == 0:
+        assert np.array_equal(host(q), ap_ref)
+    elif form == 1:
+        blk = qv.reshape(M, K // 8, 8)[:, :, [0, 2, 4, 6, 1, 3, 5, 7]] * 16
+        assert np.array_equal(host(q), blk.reshape(M, K).astype(np.int8).view(np.uint8))
+    else:
+        assert np.array_equal(host(q), e4m3_codes(qv))
+    assert np.array_equal(host(s).view(np.uint16), sa_ref.view(np.uint16))
+    xo = host(x_out).view(np.uint16)
+    assert np.array_equal(xo[:, :C], x_out_ref.view(np.uint16))
+    assert not np.any(xo[:, C:])
+
+
+def test_gather_weight_columns_exact(apex):
+    N, K = 300, 1024
+    w = synth.weights(N, K, 71)
+    ch = synth.outlier_channels(K, 72)
+    ch_d = dev(ch.astype(np.int32))
+    w_out = torch.full((N, 64), float("nan"), dtype=torch.float16, device="cuda")
+    apex.apex_gather_weight_columns(dev(w), N, K, ch_d, len(ch), w_out, 64)
+    torch.cuda.synchronize()
+    got = host(w_out).view(np.uint16)
+    assert np.array_equal(got[:, :len(ch)], np.ascontiguousarray(w[:, ch]).view(np.uint16))
+    assert not np.any(got[:, len(ch):])
+
+
+@pytest.mark.parametrize("M,N,K,C,gw", [(16, 256, 512, 5, 128), (1, 384, 1024, 11, 128),
+                                        (129, 300, 1024, 82, 128), (200, 640, 2048, 21, 512),
+                                        (256, 512, 2048, 64, 2048), (300, 1000, 1152, 130, 128)])
+def test_gemm_fp8_dual_matches_oracle(apex, M, N, K, C, gw):
+    x = synth.activations(M, K, "outlier", 80 + M)
+    w = synth.weights(N, K, 80 + N)
+    ch = np.sort(np.random.default_rng(M + C).choice(K, size=C, replace=False))
+    Cp = -(-C // 64) * 64
+    q, s, x_out, wc, sw, w_out = dual_inputs(apex, x, w, ch, Cp, gw)
+    y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+    apex.apex_w4a4_gemm_fp8_dual(M, N, K, 128, gw, q, s, wc, sw, x_out, w_out, Cp, y)
+    torch.cuda.synchronize()
+    check_status(apex)
+    x_in, x_out_ref = oracle.split_outlier_channels(x, ch)
+    ap, sa = oracle.quantize_pack(x_in, 128)
+    wp, swr = oracle.quantize_pack(w, gw)
+    ref = oracle.gemm_dual(ap, sa, wp, swr, x_out_ref, np.ascontiguousarray(w[:, ch]), M, N, K,
+                           128, gw)
+    assert_close(host(y).astype(np.float64), ref)
+
+
+def test_gemm_fp8_dual_full_size_prefill(apex):
+    """The prefill workload with its own outlier channels (1% of K, x20) through the dual
+    path; sampled rows against the oracle, and the dual path's error against the exact fp16
+    product below the plain W4A4 path's."""
+    g = synth.workloads()["prefill_m4096_n8192_k8192"]
+    a, w = synth.make(g)
+    ch = synth.outlier_channels(g.K, g.seed * 16 + 2)
+    C = len(ch)
+    Cp = -(-C // 64) * 64
+    q, s, x_out, wc, sw, w_out = dual_inputs(apex, a, w, ch, Cp)
+    y = torch.empty((g.M, g.N), dtype=torch.float16, device="cuda")
+    apex.apex_w4a4_gemm_fp8_dual(g.M, g.N, g.K, 128, 128, q, s, wc, sw, x_out, w_out, Cp, y)
+    torch.cuda.synchronize()
+    check_status(apex)
+    rows = np.array([0, 1, 127, 128, g.M // 3, g.M - 1], dtype=np.int64)
+    x_in, x_out_ref = oracle.split_outlier_channels(a[rows], ch)
+    ap, sa = oracle.quantize_pack(x_in, 128)
+    wp, swr = oracle.quantize_pack(w, 128)
+    ref = oracle.gemm_dual(ap, sa, wp, swr, x_out_ref, np.ascontiguousarray(w[:, ch]),
+                           rows.size, g.N, g.K, 128, 128)
+    got = host(y)[rows].astype(np.float64)
+    assert_close(got, ref)
+    exact = a[rows].astype(np.float64) @ w.astype(np.float64).T
+    ap1, sa1 = oracle.quantize_pack(a[rows], 128)
+    single = oracle.gemm(ap1, sa1, wp, swr, rows.size, g.N, g.K, 128, 128)
+    assert np.abs(got - exact).mean() < 0.5 * np.abs(single - exact).mean()
