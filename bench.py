@@ -171,16 +171,21 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ the apex arm
 
-WIDE_MIN_M = 128   # from this many tokens on, the step uses one-byte operand forms
+EXPANDED_MIN_M = 128   # from this many tokens on: one byte per activation (int8 path)
+FP8_MIN_M = 1024       # from this many tokens on: the E4M3-carrier GEMM (enough 128 x 256
+                       # tiles to fill the SMs at these widths)
 FORM_OVERRIDE = None   # set by --form
 
 
 def activation_form(M: int) -> str:
-    """Operand form of the step: packed int4 (few tokens: memory-bound), or E4M3 codes of the
-    same int4 values for many tokens (compute-bound; the E4M3-carrier GEMM)."""
+    """Operand form of the step: packed int4 (few tokens: memory-bound), the expanded int8
+    activations of the int8 path (a few hundred tokens), or E4M3 codes of the same int4
+    values for many tokens (compute-bound; the E4M3-carrier GEMM)."""
     if FORM_OVERRIDE:
         return FORM_OVERRIDE
-    return "fp8" if M >= WIDE_MIN_M else "packed"
+    if M >= FP8_MIN_M:
+        return "fp8"
+    return "expanded" if M >= EXPANDED_MIN_M else "packed"
 
 
 class Problem:
@@ -692,7 +697,7 @@ def chain_line(apex, torch, M, steps, warmup, world):
     up, down = synth.workloads()["mlp_up_m2048_n28672_k8192"], \
         synth.workloads()["mlp_down_m2048_n8192_k28672"]
     K, H, N = up.K, up.N, down.N
-    exp = activation_form(M) == "expanded"
+    exp = M >= EXPANDED_MIN_M   # the quantized-output epilogue belongs to the int8 path
     dev = torch.device("cuda")
     x = torch.from_numpy(synth.activations(M, K, "student_t", 7)).to(dev)
     w1 = torch.from_numpy(synth.weights(H, K, 8)).to(dev)
@@ -736,7 +741,7 @@ def chain_line(apex, torch, M, steps, warmup, world):
     u_ms = max_over_ranks(u_ms / steps, world)
     ops = 2.0 * M * K * H + 2.0 * M * H * N
     return {"sweep": f"mlp_chain_m{M}", "M": M, "K": K, "hidden": H, "N": N,
-            "activation_form": activation_form(M), "steps": steps,
+            "activation_form": "expanded" if exp else "packed", "steps": steps,
             "fused_step_ms": round(f_ms, 5), "unfused_step_ms": round(u_ms, 5),
             "fused_TOPS": round(job_throughput(ops, f_ms, world), 2),
             "unfused_TOPS": round(job_throughput(ops, u_ms, world), 2),

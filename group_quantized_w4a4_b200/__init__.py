@@ -28,6 +28,7 @@ __all__ = [
     "apex_w4a4_gemm_fp8", "apex_w4a4_group_partials_fp8", "quantize_act_fp8",
     "pack_weights_fp8", "gemm_fp8",
     "apex_gather_weight_columns", "apex_quantize_act_int4_dual", "apex_w4a4_gemm_fp8_dual",
+    "apex_select_weight_group",
     "apex_w4a4_gemm_workspace_size", "apex_w4a4_group_partials", "apex_get_device_status",
     "apex_set_wait_limit_ns", "apex_status_string", "apex_debug_withhold_step",
     "apex_debug_trace_next_gemm", "apex_debug_gemm_plan", "apex_debug_partials_split",
@@ -124,6 +125,9 @@ def load_library(build_if_missing: bool = True):
         lib.apex_set_wait_limit_ns.restype = None
         lib.apex_status_string.argtypes = [st]
         lib.apex_status_string.restype = ctypes.c_char_p
+        lib.apex_select_weight_group.argtypes = [I64, I64, I64, ctypes.c_double,
+                                                 ctypes.c_double]
+        lib.apex_select_weight_group.restype = I32
         lib.apex_debug_withhold_step.argtypes = [I32]
         lib.apex_debug_withhold_step.restype = None
         lib.apex_debug_partials_split.argtypes = [I32]
@@ -381,6 +385,12 @@ def apex_get_device_status(stream=None) -> int:
 
 def apex_set_wait_limit_ns(ns: int):
     load_library().apex_set_wait_limit_ns(int(ns))
+
+
+def apex_select_weight_group(M, N, K, rho, ridge_ops_per_byte) -> int:
+    """Host only: 128 or K, see the C header (0 for invalid arguments)."""
+    return int(load_library().apex_select_weight_group(int(M), int(N), int(K), float(rho),
+                                                       float(ridge_ops_per_byte)))
 
 
 def apex_debug_withhold_step(step: int):

@@ -503,6 +503,7 @@ apex_status_t f8_setup(int64_t M, int64_t N, int64_t K, int32_t group_w, const v
   a.G = (int)(K / 128);
   a.Gw = (int)(K / group_w);
   a.gpg = group_w / 128;
+  a.gpg_shift = (a.gpg & (a.gpg - 1)) == 0 ? __builtin_ctz((unsigned)a.gpg) : -1;
   a.tiles_m = p.tiles_m;
   a.tiles_n = p.tiles_n;
   a.T = p.T;
@@ -811,6 +812,26 @@ apex_status_t apex_debug_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t sms,
   plan[4] = p.streamk;
   plan[5] = p.cluster;
   return APEX_OK;
+}
+
+int32_t apex_select_weight_group(int64_t M, int64_t N, int64_t K, double rho,
+                                 double ridge_ops_per_byte) {
+  if (M <= 0 || N <= 0 || K <= 0 || K % 128 || !(rho > 0.0) || !(ridge_ops_per_byte > 0.0))
+    return 0;
+  // Below the ridge the weight stream bounds the GEMM and the dequantisation hides behind
+  // it: keep the finest groups.
+  const double bytes = (double)M * K / 2 + (double)N * K / 2 + 2.0 * M * (K / 128) +
+                       2.0 * N * (K / 128) + 2.0 * M * N;
+  const double intensity = 2.0 * M * N * K / bytes;
+  if (intensity < ridge_ops_per_byte) return 128;
+  // Above it, per output and per 128-wide K-group the tensor cores do 2*128 operations and
+  // the CUDA cores the dequantisation: with 128-wide weight groups one fp32 product of the
+  // two scales and one fma (4 operations), with one weight scale per row only the fma (2;
+  // the scale is applied once after the sum).  At rho times the CUDA-core rate, the
+  // dequantisation takes d * rho / 256 of the tensor time; keep 128-wide groups while that
+  // is at most half.
+  if (4.0 * rho / 256.0 <= 0.5) return 128;
+  return (int32_t)K;
 }
 
 void apex_debug_withhold_step(int32_t step) { t_withhold = step; }

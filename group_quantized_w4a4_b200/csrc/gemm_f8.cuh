@@ -55,6 +55,7 @@ struct F8Args {
   int G;             // K / 128
   int Gw;            // K / gw
   int gpg;           // K-groups per weight scale (gw / 128)
+  int gpg_shift;     // log2(gpg) when gpg is a power of two, else -1
   int tiles_m, tiles_n, T;
   int P;             // persistent CTAs (gridDim.x)
   int sa_vec;        // sa rows readable as 16-byte blocks of 8 groups
@@ -111,17 +112,12 @@ struct F8Cfg {
   static_assert(CPT % LC == 0 && (SPT == 8 || SPT == 4), "epilogue split");
 };
 
-// Tile t -> (token tile, weight tile): bands of 8 token tiles, weight tiles across each band,
-// so the CTAs running at once share both operands' tiles in L2.
+// Tile t -> (token tile, weight tile), token tiles fastest: the CTAs running at once cover all
+// token tiles of a few weight tiles, so each weight tile streams from HBM about once and is
+// read by every token tile while it is in L2 (the activations, a few tens of MB, stay in L2).
 __device__ __forceinline__ void f8_tile(const F8Args& a, int t, int& tm, int& tn) {
-  constexpr int BAND = 8;
-  const int per = BAND * a.tiles_n;
-  const int band = t / per;
-  const int first = band * BAND;
-  const int rows = min(a.tiles_m - first, BAND);
-  const int r = t - band * per;
-  tm = first + r % rows;
-  tn = r / rows;
+  tm = t % a.tiles_m;
+  tn = t / a.tiles_m;
 }
 
 // The NG (8 or 4) fp16 scales of groups g0 .. g0+NG-1 of one row (raw bits, packed two per
@@ -130,7 +126,8 @@ __device__ __forceinline__ void f8_tile(const F8Args& a, int t, int& tm, int& tn
 // scale group.
 template <int NG>
 __device__ __forceinline__ uint4 scale_block(const __half* base, int row, int rows, int ld,
-                                             int g0, int G, int gpg, bool vec) {
+                                             int g0, int G, int gpg, bool vec,
+                                             int gpg_shift = 0) {
   if (row >= rows) return make_uint4(0, 0, 0, 0);
   const __half* r = base + (size_t)row * ld;
   if (vec) {
@@ -139,9 +136,15 @@ __device__ __forceinline__ uint4 scale_block(const __half* base, int row, int ro
     return make_uint4(v.x, v.y, 0u, 0u);
   }
   uint32_t h[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  if (gpg_shift >= 0) {   // coarse groups: repeated indices, which the loads share
 #pragma unroll
-  for (int j = 0; j < NG; ++j)
-    h[j] = g0 + j < G ? (uint32_t)__half_as_ushort(r[(g0 + j) / gpg]) : 0u;
+    for (int j = 0; j < NG; ++j)
+      h[j] = g0 + j < G ? (uint32_t)__half_as_ushort(__ldg(r + ((g0 + j) >> gpg_shift))) : 0u;
+  } else {
+#pragma unroll
+    for (int j = 0; j < NG; ++j)
+      h[j] = g0 + j < G ? (uint32_t)__half_as_ushort(r[(g0 + j) / gpg]) : 0u;
+  }
   return make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
                     h[6] | (h[7] << 16));
 }
@@ -360,7 +363,7 @@ __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
                           0u);
       } else {
         return scale_block<C::SPT>(args.sw, tn * C::BN + sw_col, args.N, args.Gw, gb8 + sw_g0,
-                                   G, args.gpg, sw_vec);
+                                   G, args.gpg, sw_vec, args.gpg_shift);
       }
     };
     // the first block's scales before the first group

@@ -282,6 +282,25 @@ apex_status_t apex_debug_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t sms,
                                    int32_t with_workspace, int32_t *plan);
 
 /*
+ * The speed side of the APEX4 page's "rho-aware granularity adaptation" ("APEX4: Efficient
+ * Pure W4A4 LLM Inference via Intra-SM Compute Rebalancing", abstract: the tensor-core to
+ * CUDA-core throughput ratio rho governs the group-dequantisation bottleneck; the
+ * mixed-granularity mode recovers the high-rho GPU).  Host only, no device work.
+ *   rho:    dense integer tensor-core operations per second / fp32 CUDA-core operations per
+ *           second (the page: 8 L40S, 16 RTX 3090 and A40, 64 A100; B200: about 60-64)
+ *   ridge_ops_per_byte: tensor operations per second / HBM bytes per second
+ * Returns the weight group for an M x N x K W4A4 GEMM with 128-wide activation groups: 128
+ * when the GEMM is below the ridge (memory-bound: the dequantisation hides behind the weight
+ * stream) or when rho is low enough that the 128-wide groups' dequantisation (one scale
+ * product and one fma per partial) costs at most half of the tensor time (4*rho/256 <= 0.5);
+ * otherwise K, one weight scale per output channel (only the fma remains per partial).
+ * Returns 0 for invalid arguments (non-positive sizes or rates, K % 128 != 0).  Accuracy is
+ * not modelled (it needs trained weights); the choice is the speed side only.
+ */
+int32_t apex_select_weight_group(int64_t M, int64_t N, int64_t K, double rho,
+                                 double ridge_ops_per_byte);
+
+/*
  * Test hook: the next GEMM launch on this host thread skips the bulk copy of pipeline stage
  * `step` (two or four K-groups, counted within each CTA), so its consumers wait until the
  * time limit.  -1 turns it off.  Used only to test the timeout path; never needed by callers.
