@@ -628,9 +628,65 @@ def run_sweep(args, rank, world, local):
     for m in (2048, 16):
         line = chain_line(apex, torch, m, steps, args.warmup, world)
         lines.append(line)
+    lines.append(fp8_chain_line(apex, torch, 2048, steps, args.warmup, world))
     lines.append(dual_line(apex, torch, synth.workloads()[SECOND_WORKLOAD], steps, args.warmup,
                            world, l2, peaks, peaks_kind, int8_peak))
     return lines if rank == 0 else None
+
+
+def fp8_chain_line(apex, torch, M, steps, warmup, world):
+    """The MLP pair (8192 -> 28672 -> 8192) chained on the E4M3 path, timed as one step two
+    ways: the up layer writing the down layer's E4M3-coded activations in its epilogue
+    (apex_w4a4_gemm_fp8_quant), and unfused (fp16 output, then the E4M3 quantizer)."""
+    up, down = synth.workloads()["mlp_up_m2048_n28672_k8192"], \
+        synth.workloads()["mlp_down_m2048_n8192_k28672"]
+    K, H, N = up.K, up.N, down.N
+    dev = torch.device("cuda")
+    x = torch.from_numpy(synth.activations(M, K, "student_t", 7)).to(dev)
+    w1 = torch.from_numpy(synth.weights(H, K, 8)).to(dev)
+    w1c, w1s = apex.pack_weights_fp8(w1, 128)
+    del w1
+    w2 = torch.from_numpy(synth.weights(N, H, 9)).to(dev)
+    w2c, w2s = apex.pack_weights_fp8(w2, 128)
+    del w2
+    xa = torch.empty((M, K), dtype=torch.uint8, device=dev)
+    xs = torch.empty((M, K // 128), dtype=torch.float16, device=dev)
+    ha = torch.empty((M, H), dtype=torch.uint8, device=dev)
+    hs = torch.empty((M, H // 128), dtype=torch.float16, device=dev)
+    hy = torch.empty((M, H), dtype=torch.float16, device=dev)
+    y = torch.empty((M, N), dtype=torch.float16, device=dev)
+
+    def fused(i, s):
+        apex.apex_quantize_act_int4_fp8(x, M, K, 128, xa, xs, s)
+        apex.apex_w4a4_gemm_fp8_quant(M, H, K, 128, 128, xa, xs, w1c, w1s, None, ha, hs, s)
+        apex.apex_w4a4_gemm_fp8(M, N, H, 128, 128, ha, hs, w2c, w2s, y, s)
+
+    def unfused(i, s):
+        apex.apex_quantize_act_int4_fp8(x, M, K, 128, xa, xs, s)
+        apex.apex_w4a4_gemm_fp8(M, H, K, 128, 128, xa, xs, w1c, w1s, hy, s)
+        apex.apex_quantize_act_int4_fp8(hy, M, H, 128, ha, hs, s)
+        apex.apex_w4a4_gemm_fp8(M, N, H, 128, 128, ha, hs, w2c, w2s, y, s)
+
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        fused(i, stream)
+        unfused(i, stream)
+    torch.cuda.synchronize()
+    if apex.apex_get_device_status() != 0:
+        raise RuntimeError("device status not clean after the chain warm-up")
+    f_ms, _ = timed_graph(torch, fused, steps, warmup, world)
+    u_ms, _ = timed_graph(torch, unfused, steps, warmup, world)
+    f_ms = max_over_ranks(f_ms / steps, world)
+    u_ms = max_over_ranks(u_ms / steps, world)
+    ops = 2.0 * M * K * H + 2.0 * M * H * N
+    return {"sweep": f"mlp_chain_fp8_m{M}", "M": M, "K": K, "hidden": H, "N": N,
+            "activation_form": "fp8", "steps": steps,
+            "fused_step_ms": round(f_ms, 5), "unfused_step_ms": round(u_ms, 5),
+            "fused_TOPS": round(job_throughput(ops, f_ms, world), 2),
+            "unfused_TOPS": round(job_throughput(ops, u_ms, world), 2),
+            "what": ("x -> quantize -> up (8192 -> 28672) -> down (28672 -> 8192) on the E4M3 "
+                     "path; fused: the up layer writes the down layer's E4M3 codes and scales "
+                     "in its epilogue; unfused: fp16 output, then the quantizer")}
 
 
 def dual_line(apex, torch, g, steps, warmup, world, l2, peaks, peaks_kind, int8_peak):

@@ -28,7 +28,7 @@ __all__ = [
     "apex_w4a4_gemm_fp8", "apex_w4a4_group_partials_fp8", "quantize_act_fp8",
     "pack_weights_fp8", "gemm_fp8",
     "apex_gather_weight_columns", "apex_quantize_act_int4_dual", "apex_w4a4_gemm_fp8_dual",
-    "apex_select_weight_group",
+    "apex_select_weight_group", "apex_w4a4_gemm_fp8_quant",
     "apex_w4a4_gemm_workspace_size", "apex_w4a4_group_partials", "apex_get_device_status",
     "apex_set_wait_limit_ns", "apex_status_string", "apex_debug_withhold_step",
     "apex_debug_trace_next_gemm", "apex_debug_gemm_plan", "apex_debug_partials_split",
@@ -99,6 +99,9 @@ def load_library(build_if_missing: bool = True):
         lib.apex_unpack_int4_fp8.restype = st
         lib.apex_w4a4_gemm_fp8.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P]
         lib.apex_w4a4_gemm_fp8.restype = st
+        lib.apex_w4a4_gemm_fp8_quant.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P, P,
+                                                 P]
+        lib.apex_w4a4_gemm_fp8_quant.restype = st
         lib.apex_w4a4_group_partials_fp8.argtypes = [I64, I64, I64, P, P, P, P]
         lib.apex_w4a4_group_partials_fp8.restype = st
         lib.apex_gather_weight_columns.argtypes = [P, I64, I64, P, I32, P, I32, P]
@@ -278,6 +281,18 @@ def apex_w4a4_gemm_fp8(M, N, K, group_a, group_w, a_codes, a_scales, w_codes, w_
                                              _ptr(a_scales), _ptr(w_codes), _ptr(w_scales),
                                              _ptr(y_f16), _stream(stream)),
            "apex_w4a4_gemm_fp8")
+
+
+def apex_w4a4_gemm_fp8_quant(M, N, K, group_a, group_w, a_codes, a_scales, w_codes, w_scales,
+                             y_f16, yq_codes, yq_scales, stream=None):
+    """The E4M3-carrier GEMM plus its output quantized as the next layer's E4M3-coded
+    activations (y_f16 may be None); see the C header."""
+    _check(load_library().apex_w4a4_gemm_fp8_quant(M, N, K, group_a, group_w, _ptr(a_codes),
+                                                   _ptr(a_scales), _ptr(w_codes),
+                                                   _ptr(w_scales), _ptr(y_f16),
+                                                   _ptr(yq_codes), _ptr(yq_scales),
+                                                   _stream(stream)),
+           "apex_w4a4_gemm_fp8_quant")
 
 
 def apex_w4a4_group_partials_fp8(M, N, K, a_codes, w_codes, partials_i32, stream=None):

@@ -467,12 +467,12 @@ F8Plan make_f8_plan(int64_t M, int64_t N, int sms_override = 0) {
 #define APEX_F8_EPI_WARPS 8
 #endif
 
-template <int MODE, bool DUAL = false>
+template <int MODE, bool DUAL = false, bool QOUT = false>
 apex_status_t launch_f8(const F8Plan& p, const CUtensorMap& ma, const CUtensorMap& mb,
                         const apex::F8Args& a, cudaStream_t s, const CUtensorMap& mxo_,
                         const CUtensorMap& mwo_) {
   using C = apex::F8Cfg<APEX_F8_EPI_WARPS>;
-  auto kern = apex::w4a4_gemm_f8_kernel<MODE, APEX_F8_EPI_WARPS, DUAL>;
+  auto kern = apex::w4a4_gemm_f8_kernel<MODE, APEX_F8_EPI_WARPS, DUAL, QOUT>;
   static thread_local int attr_dev = -1;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return APEX_ERR_CUDA;
@@ -575,6 +575,36 @@ apex_status_t apex_w4a4_gemm_fp8(int64_t M, int64_t N, int64_t K, int32_t group_
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return group_w == K ? launch_f8<apex::F8_PER_CHANNEL>(p, ma, mb, a, s, ma, mb)
                       : launch_f8<apex::F8_GROUPED>(p, ma, mb, a, s, ma, mb);
+}
+
+apex_status_t apex_w4a4_gemm_fp8_quant(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                       int32_t group_w, const void* a_codes,
+                                       const void* a_scales, const void* w_codes,
+                                       const void* w_scales, void* y_f16, void* yq_codes,
+                                       void* yq_scales, void* stream) {
+  apex_status_t st = check_gemm_args(M, N, K, group_a, group_w);
+  if (st != APEX_OK) return st;
+  if (!a_scales || !w_scales || !yq_codes || !yq_scales) return APEX_ERR_INVALID_ARG;
+  if (N % 128) return APEX_ERR_UNSUPPORTED;   // every 128 outputs are one next-layer group
+  if (!aligned(a_scales, 2) || !aligned(w_scales, 2) || (y_f16 && !aligned(y_f16, 2)) ||
+      !aligned(yq_codes, 16) || !aligned(yq_scales, 2))
+    return APEX_ERR_ALIGNMENT;
+  F8Plan p;
+  apex::F8Args a;
+  CUtensorMap ma, mb;
+  st = f8_setup(M, N, K, group_w, a_codes, w_codes, p, a, ma, mb);
+  if (st != APEX_OK) return st;
+  a.sa = static_cast<const __half*>(a_scales);
+  a.sw = static_cast<const __half*>(w_scales);
+  a.y = static_cast<__half*>(y_f16);
+  a.qout = static_cast<uint8_t*>(yq_codes);
+  a.qscale = static_cast<__half*>(yq_scales);
+  a.sa_vec = a.G % 8 == 0 && aligned(a_scales, 16);
+  a.sw_vec = group_w == 128 && a.G % 8 == 0 && aligned(w_scales, 16);
+  a.y_vec = y_f16 && N % 8 == 0 && aligned(y_f16, 16);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return group_w == K ? launch_f8<apex::F8_PER_CHANNEL, false, true>(p, ma, mb, a, s, ma, mb)
+                      : launch_f8<apex::F8_GROUPED, false, true>(p, ma, mb, a, s, ma, mb);
 }
 
 apex_status_t apex_w4a4_group_partials_fp8(int64_t M, int64_t N, int64_t K, const void* a_codes,

@@ -42,6 +42,7 @@
 #include <stdint.h>
 
 #include "ptx.cuh"
+#include "quantize.cuh"
 
 namespace apex {
 
@@ -66,6 +67,10 @@ struct F8Args {
   __half* y;         // [M][N]
   int32_t* dump;     // [G][M][N] per-group partials (export kernel only)
   unsigned long long wait_ns;
+  // Optional quantized output (QOUT instantiations): Y's fp16 values quantized as the next
+  // layer's activations, E4M3 codes [M][N] and fp16 scales [M][N/128].  y may then be null.
+  uint8_t* qout;
+  __half* qscale;
   // The outlier dual path (0: none): NO extra K-steps of 64 fp16 channels per tile, from the
   // maps tmXo (x_out [M][64*NO]) and tmWo (w_out [N][64*NO]), multiplied by kind::f16 MMAs
   // and added with unit scale after the 4-bit groups.
@@ -180,7 +185,8 @@ __device__ __forceinline__ uint32_t half2_bits(float2 v) {
 
 
 // DUAL: the outlier dual path's K-steps are compiled in (args.NO of them; else none).
-template <int MODE, int EW, bool DUAL = false>
+// QOUT: the output is also quantized as the next layer's E4M3-coded activations.
+template <int MODE, int EW, bool DUAL = false, bool QOUT = false>
 __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
     w4a4_gemm_f8_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -532,7 +538,7 @@ __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
         }
         // the finished tile: this thread's token row, 128 consecutive outputs (after a wait
         // that gave up, nothing: the next block barrier takes the decision to stop)
-        if (ok && m < args.M) {
+        if (ok && m < args.M && args.y != nullptr) {
           __half* dst = args.y + (size_t)m * args.N + n0;
           if (args.y_vec && n0 + C::CPT <= args.N) {
 #pragma unroll
@@ -546,6 +552,33 @@ __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
               const float v = (e & 1) ? acc[e / 2].y : acc[e / 2].x;
               if (n0 + e < args.N) dst[e] = __float2half_rn(v);
             }
+          }
+        }
+        if constexpr (QOUT) {
+          // The next layer's activations: this thread's 128 outputs of token m are exactly one
+          // 128-wide K-group of that token's input to the next layer (N % 128 == 0), so the
+          // group's scale and E4M3 codes are made here, from the fp16 values Y holds and with
+          // the activation quantizer's own rule; no other thread is involved.  (A tile's
+          // upper half may lie past N: N % 128 == 0, so n0 < N means all 128 are inside.)
+          if (ok && m < args.M && n0 < args.N) {
+            float amax = 0.0f;
+#pragma unroll
+            for (int e = 0; e < C::CPT / 2; ++e)
+              amax = fmaxf(amax, fmaxf(fabsf(acc[e].x), fabsf(acc[e].y)));
+            // rounding to fp16 is monotonic: the largest |fp16(v)| is fp16(largest |v|)
+            const __half sc = group_scale(__half2float(__float2half_rn(amax)));
+            const QScale qs = make_qscale(__half2float(sc));
+            uint8_t* qd = args.qout + (size_t)m * args.N + n0;
+#pragma unroll
+            for (int e = 0; e < C::CPT / 2; e += 8) {
+              const uint4 h0 = make_uint4(half2_bits(acc[e]), half2_bits(acc[e + 1]),
+                                          half2_bits(acc[e + 2]), half2_bits(acc[e + 3]));
+              const uint4 h1 = make_uint4(half2_bits(acc[e + 4]), half2_bits(acc[e + 5]),
+                                          half2_bits(acc[e + 6]), half2_bits(acc[e + 7]));
+              const uint2 c0 = quant_e4m3_8(h0, qs), c1 = quant_e4m3_8(h1, qs);
+              *reinterpret_cast<uint4*>(qd + 2 * e) = make_uint4(c0.x, c0.y, c1.x, c1.y);
+            }
+            args.qscale[(size_t)m * (args.N / 128) + n0 / 128] = sc;
           }
         }
       }

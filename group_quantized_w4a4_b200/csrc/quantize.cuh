@@ -68,14 +68,16 @@ __device__ __forceinline__ int quant1(float f, const QScale& qs) {
 }
 
 // Two integer-valued floats (|v| <= 8) as E4M3 codes, exact: lo in bits 0..7, hi in 8..15.
-// A zero is always coded +0 (0x00): q = 0 reached from a negative value is -0.0 in fp32,
-// and adding +0 turns it into +0 (IEEE round to nearest).
 __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
-      : "=h"(r)
-      : "f"(__fadd_rn(hi, 0.0f)), "f"(__fadd_rn(lo, 0.0f)));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Four E4M3 codes with every negative zero (0x80, from a q = 0 reached by rounding a
+// negative value) replaced by +0 (0x00): a zero is always coded 0x00.
+__device__ __forceinline__ uint32_t e4m3_plus_zero(uint32_t w) {
+  return w & ~__vcmpeq4(w, 0x80808080u);
 }
 
 // The same 8 values as the E4M3 codes of q (one byte per element, in element order): the
@@ -87,8 +89,8 @@ __device__ __forceinline__ uint2 quant_e4m3_8(const uint4& v, const QScale& qs) 
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const float2 a = __half22float2(h[2 * i]), b = __half22float2(h[2 * i + 1]);
-    w[i] = e4m3x2(quant1f(a.x, qs), quant1f(a.y, qs)) |
-           (e4m3x2(quant1f(b.x, qs), quant1f(b.y, qs)) << 16);
+    w[i] = e4m3_plus_zero(e4m3x2(quant1f(a.x, qs), quant1f(a.y, qs)) |
+                          (e4m3x2(quant1f(b.x, qs), quant1f(b.y, qs)) << 16));
   }
   return make_uint2(w[0], w[1]);
 }

@@ -237,6 +237,22 @@ apex_status_t apex_w4a4_gemm_fp8(int64_t M, int64_t N, int64_t K, int32_t group_
                                  void *stream);
 
 /*
+ * The E4M3-carrier GEMM whose output is also quantized as the next layer's activations (a
+ * chain of W4A4 layers without a separate quantizer pass): the computation and rules of
+ * apex_w4a4_gemm_fp8, and additionally
+ *   yq_codes [M][N] E4M3 codes, yq_scales [M][N/128] fp16:
+ * exactly what apex_quantize_act_int4_fp8 (group_a = 128) would make from the fp16 Y this
+ * call computes -- each tile holds every 128 outputs of a token that form one K-group of the
+ * next layer.  y_f16 may be NULL (then only the quantized output is written).  N % 128 == 0
+ * (APEX_ERR_UNSUPPORTED otherwise); yq_codes 16-byte, yq_scales 2-byte aligned.
+ */
+apex_status_t apex_w4a4_gemm_fp8_quant(int64_t M, int64_t N, int64_t K, int32_t group_a,
+                                       int32_t group_w, const void *a_codes,
+                                       const void *a_scales, const void *w_codes,
+                                       const void *w_scales, void *y_f16, void *yq_codes,
+                                       void *yq_scales, void *stream);
+
+/*
  * Parity export of the E4M3-carrier GEMM: every exact per-group partial, as
  * apex_w4a4_group_partials, computed by the same tensor-core path as apex_w4a4_gemm_fp8
  * (its fp32 partials stored as int32).

@@ -353,3 +353,75 @@ def test_gemm_fp8_dual_full_size_prefill(apex):
     ap1, sa1 = oracle.quantize_pack(a[rows], 128)
     single = oracle.gemm(ap1, sa1, wp, swr, rows.size, g.N, g.K, 128, 128)
     assert np.abs(got - exact).mean() < 0.5 * np.abs(single - exact).mean()
+
+
+# ------------------------------------------------------------------ quantized output
+
+
+def codes_to_q(codes):
+    """E4M3 codes of integers -> int64 values (torch's float8_e4m3fn decoding)."""
+    t = torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn)
+    return t.to(torch.float32).numpy().astype(np.int64)
+
+
+@pytest.mark.parametrize("M,N,K,gw", [(16, 256, 512, 128), (1, 128, 128, 128),
+                                      (129, 384, 1024, 128), (300, 1024, 1152, 384),
+                                      (200, 640, 2048, 2048), (1100, 2048, 1024, 128)])
+def test_gemm_fp8_quantized_output_is_the_quantizer_of_y(apex, M, N, K, gw):
+    """The fused output equals the oracle's activation quantizer applied to the fp16 Y the
+    same call wrote, as E4M3 codes and fp16 scales, bit for bit; Y meets the GEMM bar; and
+    without Y the quantized output is the same."""
+    x = synth.activations(M, K, "outlier", 60 + M)
+    w = synth.weights(N, K, 60 + N)
+    ac, sa = apex.quantize_act_fp8(dev(x), 128)
+    wc, sw = apex.pack_weights_fp8(dev(w), gw)
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    yq = torch.empty((M, N), dtype=torch.uint8, device="cuda")
+    ys = torch.empty((M, N // 128), dtype=torch.float16, device="cuda")
+    apex.apex_w4a4_gemm_fp8_quant(M, N, K, 128, gw, ac, sa, wc, sw, y, yq, ys)
+    torch.cuda.synchronize()
+    check_status(apex)
+    ap, sar = oracle.quantize_pack(x, 128)
+    wp, swr = oracle.quantize_pack(w, gw)
+    y_h = host(y)
+    assert_close(y_h.astype(np.float64), oracle.gemm(ap, sar, wp, swr, M, N, K, 128, gw))
+    q_ref, s_ref = oracle.quantize_pack(y_h, 128)
+    assert np.array_equal(host(yq), e4m3_codes(oracle.unpack(q_ref, N)))
+    assert np.array_equal(host(ys).view(np.uint16), s_ref.view(np.uint16))
+    yq2, ys2 = torch.zeros_like(yq), torch.zeros_like(ys)
+    apex.apex_w4a4_gemm_fp8_quant(M, N, K, 128, gw, ac, sa, wc, sw, None, yq2, ys2)
+    torch.cuda.synchronize()
+    check_status(apex)
+    assert torch.equal(yq2, yq) and torch.equal(ys2, ys)
+
+
+def test_fp8_chained_layers_through_the_quantized_output(apex):
+    """Two W4A4 layers on the E4M3 path, the first one's quantized output fed straight to the
+    second: the second's result equals the oracle GEMM on the operands the first produced."""
+    M, K, H, N = 256, 1024, 2048, 512
+    x = synth.activations(M, K, "student_t", 223)
+    w1, w2 = synth.weights(H, K, 224), synth.weights(N, H, 225)
+    ac, sa = apex.quantize_act_fp8(dev(x), 128)
+    w1c, w1s = apex.pack_weights_fp8(dev(w1), 128)
+    w2c, w2s = apex.pack_weights_fp8(dev(w2), 128)
+    hq = torch.empty((M, H), dtype=torch.uint8, device="cuda")
+    hs = torch.empty((M, H // 128), dtype=torch.float16, device="cuda")
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    apex.apex_w4a4_gemm_fp8_quant(M, H, K, 128, 128, ac, sa, w1c, w1s, None, hq, hs)
+    apex.apex_w4a4_gemm_fp8(M, N, H, 128, 128, hq, hs, w2c, w2s, y)
+    torch.cuda.synchronize()
+    check_status(apex)
+    w2p, w2sr = oracle.quantize_pack(w2, 128)
+    ref = oracle.gemm(pack(codes_to_q(host(hq))), host(hs), w2p, w2sr, M, N, H, 128, 128)
+    assert_close(host(y).astype(np.float64), ref)
+
+
+def test_gemm_fp8_quant_argument_rules(apex):
+    t = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
+    h = torch.zeros(1 << 10, dtype=torch.float16, device="cuda")
+    with pytest.raises(apex.ApexError) as e:      # N not a multiple of 128
+        apex.apex_w4a4_gemm_fp8_quant(16, 200, 256, 128, 128, t, h, t, h, None, t, h)
+    assert e.value.code == apex.APEX_ERR_UNSUPPORTED
+    with pytest.raises(apex.ApexError) as e:      # no quantized output buffer
+        apex.apex_w4a4_gemm_fp8_quant(16, 256, 256, 128, 128, t, h, t, h, None, None, h)
+    assert e.value.code == apex.APEX_ERR_INVALID_ARG
