@@ -116,3 +116,62 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros((4, 256), dtype=torch.float16)
     with pytest.raises((ValueError, RuntimeError)):
         apex.quantize_act(x)
+
+
+def test_fp8_path_argument_errors_are_host_side(lib):
+    def g(M=16, N=256, K=256, ga=128, gw=128, a=0x1000, sa=0x2000, w=0x3000, sw=0x4000,
+          y=0x5000):
+        return lib.apex_w4a4_gemm_fp8(M, N, K, ga, gw, P(a), P(sa), P(w), P(sw), P(y), None)
+    assert g(K=200) == apex.APEX_ERR_INVALID_ARG
+    assert g(ga=64) == apex.APEX_ERR_UNSUPPORTED
+    assert g(a=0) == apex.APEX_ERR_INVALID_ARG
+    assert g(y=0) == apex.APEX_ERR_INVALID_ARG
+    assert g(a=0x1008) == apex.APEX_ERR_ALIGNMENT       # TMA base: 16 bytes
+    assert g(w=0x3004) == apex.APEX_ERR_ALIGNMENT
+    assert g(sa=0x2001) == apex.APEX_ERR_ALIGNMENT
+
+    def gq(N=256, y=None, yq=0x6000, yqs=0x7000):
+        return lib.apex_w4a4_gemm_fp8_quant(16, N, 256, 128, 128, P(0x1000), P(0x2000),
+                                            P(0x3000), P(0x4000), P(y), P(yq), P(yqs), None)
+    assert gq(N=200) == apex.APEX_ERR_UNSUPPORTED
+    assert gq(yq=None) == apex.APEX_ERR_INVALID_ARG
+    assert gq(yq=0x6008) == apex.APEX_ERR_ALIGNMENT
+    assert gq(y=0x5001) == apex.APEX_ERR_ALIGNMENT
+
+    q = lib.apex_quantize_act_int4_fp8
+    assert q(P(0x1000), 4, 256, 256, P(0x2000), P(0x3000), None) == apex.APEX_ERR_UNSUPPORTED
+    assert q(P(0x1000), 4, 200, 128, P(0x2000), P(0x3000), None) == apex.APEX_ERR_INVALID_ARG
+    assert q(P(0x1000), 4, 256, 128, P(0x2004), P(0x3000), None) == apex.APEX_ERR_ALIGNMENT
+    pw = lib.apex_pack_weights_int4_fp8
+    assert pw(P(0x1000), 4, 512, 96, P(0x2000), P(0x3000), None) == apex.APEX_ERR_INVALID_ARG
+    u = lib.apex_unpack_int4_fp8
+    assert u(P(0x1000), 4, 200, P(0x2000), None) == apex.APEX_ERR_INVALID_ARG    # K % 16
+    assert u(P(0x1000), 4, 256, P(0x2008), None) == apex.APEX_ERR_ALIGNMENT
+    pp = lib.apex_w4a4_group_partials_fp8
+    assert pp(4, 8, 256, P(0x1000), P(0x2000), None, None) == apex.APEX_ERR_INVALID_ARG
+
+
+def test_dual_path_argument_errors_are_host_side(lib):
+    ch = P(0x8000)
+
+    def dq(C=5, Cp=64, form=2, x=0x1000, xo=0x9000):
+        return lib.apex_quantize_act_int4_dual(P(x), 4, 256, 128, ch, C, form, P(0x2000),
+                                               P(0x3000), P(xo), Cp, None)
+    assert dq(Cp=48) == apex.APEX_ERR_INVALID_ARG        # Cp % 64
+    assert dq(C=65) == apex.APEX_ERR_INVALID_ARG         # C > Cp
+    assert dq(C=0) == apex.APEX_ERR_INVALID_ARG
+    assert dq(form=3) == apex.APEX_ERR_INVALID_ARG
+    assert dq(x=0x1008) == apex.APEX_ERR_ALIGNMENT
+    assert dq(xo=0x9008) == apex.APEX_ERR_ALIGNMENT
+    gw = lib.apex_gather_weight_columns
+    assert gw(P(0x1000), 8, 256, ch, 5, P(0x9000), 32, None) == apex.APEX_ERR_INVALID_ARG
+    assert gw(P(0x1000), 8, 256, ch, 5, P(0x9008), 64, None) == apex.APEX_ERR_ALIGNMENT
+
+    def dg(Cp=64, xo=0x9000):
+        return lib.apex_w4a4_gemm_fp8_dual(16, 256, 256, 128, 128, P(0x1000), P(0x2000),
+                                           P(0x3000), P(0x4000), P(xo), P(0xA000), Cp,
+                                           P(0x5000), None)
+    assert dg(Cp=0) == apex.APEX_ERR_INVALID_ARG
+    assert dg(Cp=96) == apex.APEX_ERR_INVALID_ARG
+    assert dg(Cp=512) == apex.APEX_ERR_INVALID_ARG       # more outlier channels than K
+    assert dg(xo=0x9008) == apex.APEX_ERR_ALIGNMENT
