@@ -335,6 +335,35 @@ void attach_workspace(const Plan& p, GemmArgs& a, void* ws) {
   a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + counters_bytes(p));
 }
 
+// Units (row, group) each half-warp of the 128-wide-group quantizer takes per round once a
+// batch is large enough that the loads in flight, not the per-unit latency, set its time.
+constexpr int kQuantUnitsPerRound = 2;
+constexpr int64_t kQuantBatchMinUnits = 1 << 15;
+
+template <int CH, int FORM, int UPT>
+cudaError_t quantize_launch_t(int64_t units, cudaStream_t s, const __half* xh, int64_t rows,
+                              int64_t K, int32_t group, uint8_t* pk, __half* sc, int g_shift) {
+  // 128-thread blocks: one fits on an SM next to a GEMM CTA (registers), so the GEMM that
+  // follows can start its prologue on every SM while the quantizer still runs
+  const int threads = 128;
+  const int64_t warps_needed = (units + 2 * UPT - 1) / (2 * UPT);
+  int64_t blocks = (warps_needed * 32 + threads - 1) / threads;
+  const int64_t cap = (int64_t)dev_info().sms * 32;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return launch_pdl(apex::quantize_pack_kernel<CH, FORM, UPT>, (unsigned)blocks, threads, 0, s,
+                    xh, rows, K, group, pk, sc, g_shift);
+}
+
+template <int FORM>
+cudaError_t quantize_launch_g128(int64_t units, cudaStream_t s, const __half* xh, int64_t rows,
+                                 int64_t K, uint8_t* pk, __half* sc, int g_shift) {
+  if (units >= kQuantBatchMinUnits)
+    return quantize_launch_t<1, FORM, kQuantUnitsPerRound>(units, s, xh, rows, K, 128, pk, sc,
+                                                           g_shift);
+  return quantize_launch_t<1, FORM, 1>(units, s, xh, rows, K, 128, pk, sc, g_shift);
+}
+
 apex_status_t quantize_launch(const void* x, int64_t rows, int64_t K, int32_t group, void* packed,
                               void* scales, void* stream, bool expanded = false,
                               bool e4m3 = false) {
@@ -344,41 +373,31 @@ apex_status_t quantize_launch(const void* x, int64_t rows, int64_t K, int32_t gr
     return APEX_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t units = rows * (K / group);
-  // 128-thread blocks: one fits on an SM next to a GEMM CTA (registers), so the GEMM that
-  // follows can start its prologue on every SM while the quantizer still runs
-  const int threads = 128;
-  const int64_t warps_needed = (units + 1) / 2;
-  int64_t blocks = (warps_needed * 32 + threads - 1) / threads;
-  const int64_t cap = (int64_t)dev_info().sms * 32;
-  if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
+  if (units >= (1ll << 31)) return APEX_ERR_UNSUPPORTED;   // the kernel indexes units in 32 bits
+  const int64_t gpr = K / group;                             // groups per row
+  const int g_shift = (gpr & (gpr - 1)) == 0 ? __builtin_ctzll((unsigned long long)gpr) : -1;
   const __half* xh = static_cast<const __half*>(x);
   uint8_t* pk = static_cast<uint8_t*>(packed);
   __half* sc = static_cast<__half*>(scales);
-  const unsigned nb = (unsigned)blocks;
   cudaError_t e;
   if (e4m3) {
     if (group == 128)
-      e = launch_pdl(apex::quantize_pack_kernel<1, apex::FORM_E4M3>, nb, threads, 0, s, xh, rows,
-                     K, group, pk, sc);
+      e = quantize_launch_g128<apex::FORM_E4M3>(units, s, xh, rows, K, pk, sc, g_shift);
     else if (group == 512)
-      e = launch_pdl(apex::quantize_pack_kernel<4, apex::FORM_E4M3>, nb, threads, 0, s, xh, rows,
-                     K, group, pk, sc);
+      e = quantize_launch_t<4, apex::FORM_E4M3, 1>(units, s, xh, rows, K, group, pk, sc, g_shift);
     else
-      e = launch_pdl(apex::quantize_pack_kernel<0, apex::FORM_E4M3>, nb, threads, 0, s, xh, rows,
-                     K, group, pk, sc);
+      e = quantize_launch_t<0, apex::FORM_E4M3, 1>(units, s, xh, rows, K, group, pk, sc, g_shift);
   } else if (expanded) {
     if (group != 128) return APEX_ERR_UNSUPPORTED;
-    e = launch_pdl(apex::quantize_pack_kernel<1, apex::FORM_EXPANDED>, nb, threads, 0, s, xh,
-                   rows, K, group, pk, sc);
+    e = quantize_launch_g128<apex::FORM_EXPANDED>(units, s, xh, rows, K, pk, sc, g_shift);
   } else if (group == 128) {
-    e = launch_pdl(apex::quantize_pack_kernel<1>, nb, threads, 0, s, xh, rows, K, group, pk, sc);
+    e = quantize_launch_g128<apex::FORM_PACKED>(units, s, xh, rows, K, pk, sc, g_shift);
   } else if (group == 256) {
-    e = launch_pdl(apex::quantize_pack_kernel<2>, nb, threads, 0, s, xh, rows, K, group, pk, sc);
+    e = quantize_launch_t<2, apex::FORM_PACKED, 1>(units, s, xh, rows, K, group, pk, sc, g_shift);
   } else if (group == 512) {
-    e = launch_pdl(apex::quantize_pack_kernel<4>, nb, threads, 0, s, xh, rows, K, group, pk, sc);
+    e = quantize_launch_t<4, apex::FORM_PACKED, 1>(units, s, xh, rows, K, group, pk, sc, g_shift);
   } else {
-    e = launch_pdl(apex::quantize_pack_kernel<0>, nb, threads, 0, s, xh, rows, K, group, pk, sc);
+    e = quantize_launch_t<0, apex::FORM_PACKED, 1>(units, s, xh, rows, K, group, pk, sc, g_shift);
   }
   if (e != cudaSuccess) return APEX_ERR_CUDA;
   return cuda_status(cudaPeekAtLastError());

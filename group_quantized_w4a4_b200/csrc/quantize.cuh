@@ -135,53 +135,85 @@ __device__ __forceinline__ void store_quantized(uint32_t* dst, uint2* xdst, cons
 // CH > 0: the group is exactly CH 128-wide chunks, kept in registers (one pass over HBM).
 // CH == 0: any group width; absmax pass then quantize pass (the second pass hits L2).
 // FORM: the output form (QForm).
-template <int CH, int FORM = FORM_PACKED>
+// Each half-warp takes UPT (row, group) units per round, all their loads issued before any
+// arithmetic, so that several 16-byte loads per thread are in flight (the kernel is bound by
+// memory latency, not by its arithmetic).  Units are indexed in 32 bits (the host launches
+// this kernel only when rows * K / group < 2^31) and split into (row, group) by a shift when
+// the groups per row are a power of two (g_shift >= 0).
+template <int CH, int FORM = FORM_PACKED, int UPT = 1>
 __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __restrict__ x,
                                                             int64_t rows, int64_t K, int group,
                                                             uint8_t* __restrict__ packed,
-                                                            __half* __restrict__ scales) {
+                                                            __half* __restrict__ scales,
+                                                            int g_shift) {
   // launched as a programmatic dependent: nothing is read or written before the previous
   // grid in the stream has completed
   grid_dep_wait();
   grid_dep_launch();
-  const int64_t G = K / group;
-  const int64_t units = rows * G;
+  const uint32_t G = (uint32_t)(K / group);
+  const uint32_t units = (uint32_t)(rows * G);
   const int chunks = group / 128;
   const int lane16 = threadIdx.x & 15;
-  const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t warps_total = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const uint32_t warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t warps_total = (gridDim.x * blockDim.x) >> 5;
   const int half = (threadIdx.x >> 4) & 1;
+  auto split = [&](uint32_t unit, uint32_t& row, uint32_t& g) {
+    if (g_shift >= 0) {
+      row = unit >> g_shift;
+      g = unit & (G - 1);
+    } else {
+      row = unit / G;
+      g = unit - row * G;
+    }
+  };
 
   // Warp-uniform loop: both half-warps iterate together so the shuffles stay converged.
-  for (int64_t base = warp_global * 2; base < units; base += warps_total * 2) {
-    const int64_t unit = base + half;
-    const bool live = unit < units;
-    const int64_t row = live ? unit / G : 0;
-    const int64_t g = live ? unit % G : 0;
-    const uint4* src = reinterpret_cast<const uint4*>(x + row * K + g * group) + lane16;
-    uint32_t* dst =
-        reinterpret_cast<uint32_t*>(packed + row * (K / 2) + g * (group / 2)) + lane16;
-    uint2* xdst = reinterpret_cast<uint2*>(packed + row * K + (int64_t)g * group) + lane16;
-
-    float amax = 0.0f;
+  for (uint32_t base = warp_global * 2 * UPT; base < units; base += warps_total * 2 * UPT) {
     if constexpr (CH > 0) {
-      uint4 v[CH];
+      uint4 v[UPT][CH];
+      uint32_t row[UPT], g[UPT];
+      bool live[UPT];
 #pragma unroll
-      for (int c = 0; c < CH; ++c) {
-        v[c] = live ? __ldg(src + c * 16) : make_uint4(0, 0, 0, 0);
-        amax = fmaxf(amax, absmax8(v[c]));
+      for (int u = 0; u < UPT; ++u) {
+        const uint32_t unit = base + 2 * u + half;
+        live[u] = unit < units;
+        split(live[u] ? unit : 0u, row[u], g[u]);
+        const uint4* src =
+            reinterpret_cast<const uint4*>(x + (int64_t)row[u] * K + (int64_t)g[u] * group) +
+            lane16;
+#pragma unroll
+        for (int c = 0; c < CH; ++c)
+          v[u][c] = live[u] ? __ldg(src + c * 16) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int off = 8; off >= 1; off >>= 1)
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-      const __half s = group_scale(amax);
-      const QScale qs = make_qscale(__half2float(s));
-      if (live) {
+      for (int u = 0; u < UPT; ++u) {
+        float amax = 0.0f;
 #pragma unroll
-        for (int c = 0; c < CH; ++c) store_quantized<FORM>(dst + c * 16, xdst + c * 16, v[c], qs);
-        if (lane16 == 0) scales[row * G + g] = s;
+        for (int c = 0; c < CH; ++c) amax = fmaxf(amax, absmax8(v[u][c]));
+#pragma unroll
+        for (int off = 8; off >= 1; off >>= 1)
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        const __half s = group_scale(amax);
+        const QScale qs = make_qscale(__half2float(s));
+        if (live[u]) {
+          uint32_t* dst = reinterpret_cast<uint32_t*>(packed + (int64_t)row[u] * (K / 2) +
+                                                      (int64_t)g[u] * (group / 2)) + lane16;
+          uint2* xdst = reinterpret_cast<uint2*>(packed + (int64_t)row[u] * K +
+                                                 (int64_t)g[u] * group) + lane16;
+#pragma unroll
+          for (int c = 0; c < CH; ++c)
+            store_quantized<FORM>(dst + c * 16, xdst + c * 16, v[u][c], qs);
+          if (lane16 == 0) scales[(int64_t)row[u] * G + g[u]] = s;
+        }
       }
     } else {
+      const uint32_t unit = base + half;
+      const bool live = unit < units;
+      uint32_t row, g;
+      split(live ? unit : 0u, row, g);
+      const uint4* src =
+          reinterpret_cast<const uint4*>(x + (int64_t)row * K + (int64_t)g * group) + lane16;
+      float amax = 0.0f;
       for (int c = 0; c < chunks; ++c) {
         uint4 v = live ? __ldg(src + c * 16) : make_uint4(0, 0, 0, 0);
         amax = fmaxf(amax, absmax8(v));
@@ -192,9 +224,13 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __rest
       const __half s = group_scale(amax);
       const QScale qs = make_qscale(__half2float(s));
       if (live) {
+        uint32_t* dst = reinterpret_cast<uint32_t*>(packed + (int64_t)row * (K / 2) +
+                                                    (int64_t)g * (group / 2)) + lane16;
+        uint2* xdst =
+            reinterpret_cast<uint2*>(packed + (int64_t)row * K + (int64_t)g * group) + lane16;
         for (int c = 0; c < chunks; ++c)
           store_quantized<FORM>(dst + c * 16, xdst + c * 16, __ldg(src + c * 16), qs);
-        if (lane16 == 0) scales[row * G + g] = s;
+        if (lane16 == 0) scales[(int64_t)row * G + g] = s;
       }
     }
   }
