@@ -336,11 +336,13 @@ void attach_workspace(const Plan& p, GemmArgs& a, void* ws) {
 }
 
 // Units (row, group) each half-warp of the 128-wide-group quantizer takes per round once a
-// batch is large enough that the loads in flight, not the per-unit latency, set its time.
+// batch is large enough that the loads in flight, not the per-unit latency, set its time;
+// such batches also take the fast per-value path (measured: it loses ~0.1 us on a 16-token
+// batch, where one short chain per thread is the whole time, and wins 10-25 % from 512 on).
 constexpr int kQuantUnitsPerRound = 2;
 constexpr int64_t kQuantBatchMinUnits = 1 << 15;
 
-template <int CH, int FORM, int UPT>
+template <int CH, int FORM, int UPT, bool FAST = true>
 cudaError_t quantize_launch_t(int64_t units, cudaStream_t s, const __half* xh, int64_t rows,
                               int64_t K, int32_t group, uint8_t* pk, __half* sc, int g_shift) {
   // 128-thread blocks: one fits on an SM next to a GEMM CTA (registers), so the GEMM that
@@ -351,7 +353,7 @@ cudaError_t quantize_launch_t(int64_t units, cudaStream_t s, const __half* xh, i
   const int64_t cap = (int64_t)dev_info().sms * 32;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  return launch_pdl(apex::quantize_pack_kernel<CH, FORM, UPT>, (unsigned)blocks, threads, 0, s,
+  return launch_pdl(apex::quantize_pack_kernel<CH, FORM, UPT, FAST>, (unsigned)blocks, threads, 0, s,
                     xh, rows, K, group, pk, sc, g_shift);
 }
 
@@ -361,7 +363,7 @@ cudaError_t quantize_launch_g128(int64_t units, cudaStream_t s, const __half* xh
   if (units >= kQuantBatchMinUnits)
     return quantize_launch_t<1, FORM, kQuantUnitsPerRound>(units, s, xh, rows, K, 128, pk, sc,
                                                            g_shift);
-  return quantize_launch_t<1, FORM, 1>(units, s, xh, rows, K, 128, pk, sc, g_shift);
+  return quantize_launch_t<1, FORM, 1, false>(units, s, xh, rows, K, 128, pk, sc, g_shift);
 }
 
 apex_status_t quantize_launch(const void* x, int64_t rows, int64_t K, int32_t group, void* packed,

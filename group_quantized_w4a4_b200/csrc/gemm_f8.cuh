@@ -593,30 +593,8 @@ __global__ void __launch_bounds__(F8Cfg<EW>::THREADS, 1)
   }
 }
 
-// Packed int4 [rows][K/2] -> E4M3 codes of the same q [rows][K] (element order).  Each thread
-// turns 8 packed bytes into 16 codes with byte-permute table lookups: the codes of q = 0..7
-// and of q = -8..-1 are two 8-byte tables, a nibble's low three bits index both and its sign
-// bit picks one.
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
-}
-
-// E4M3 codes of the four nibbles in the low 16 bits of w (nibble i -> byte i).
-__device__ __forceinline__ uint32_t e4m3_of_nibbles(uint32_t w) {
-  // E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits) of 0..7 and of -8..-1
-  constexpr uint32_t P0 = 0x44403800u, P1 = 0x4E4C4A48u;   // 0, 1, 2, 3 | 4, 5, 6, 7
-  constexpr uint32_t N0 = 0xCACCCED0u, N1 = 0xB8C0C4C8u;   // -8,-7,-6,-5 | -4,-3,-2,-1
-  const uint32_t idx = w & 0x7777u;
-  const uint32_t pos = prmt(P0, P1, idx);
-  const uint32_t neg = prmt(N0, N1, idx);
-  // 0xFF in byte i where nibble i is negative: selector 0xC (sign of byte 4 = 0x80) or 0x0
-  const uint32_t s = w & 0x8888u;
-  const uint32_t mask = prmt(0u, 0x80u, s | (s >> 1));
-  return (neg & mask) | (pos & ~mask);
-}
-
+// Packed int4 [rows][K/2] -> E4M3 codes of the same q [rows][K] (element order): each thread
+// turns 8 packed bytes into 16 codes (e4m3_of_nibbles, quantize.cuh).
 __global__ void __launch_bounds__(256) unpack_e4m3_kernel(const uint8_t* __restrict__ packed,
                                                          int64_t words, uint8_t* __restrict__ codes) {
   grid_dep_wait();

@@ -67,37 +67,31 @@ __device__ __forceinline__ int quant1(float f, const QScale& qs) {
   return __float2int_rn(quant1f(f, qs));
 }
 
-// Two integer-valued floats (|v| <= 8) as E4M3 codes, exact: lo in bits 0..7, hi in 8..15.
-__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
+// Byte permute: byte i of the result is byte sel[4i+3:4i] of the 8 bytes {b, a} (a = 0..3).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
 }
 
-// Four E4M3 codes with every negative zero (0x80, from a q = 0 reached by rounding a
-// negative value) replaced by +0 (0x00): a zero is always coded 0x00.
-__device__ __forceinline__ uint32_t e4m3_plus_zero(uint32_t w) {
-  return w & ~__vcmpeq4(w, 0x80808080u);
+// E4M3 codes of the four nibbles (int4 two's complement) in the low 16 bits of w, nibble i
+// -> byte i, by two 8-byte table lookups: the codes of q = 0..7 and of q = -8..-1, indexed by
+// the nibble's low three bits, the sign bit choosing the table.  E4M3: 1 sign bit, 4
+// exponent bits with bias 7, 3 mantissa bits; every q in [-8, 7] is exact and 0 is 0x00.
+__device__ __forceinline__ uint32_t e4m3_of_nibbles(uint32_t w) {
+  constexpr uint32_t P0 = 0x44403800u, P1 = 0x4E4C4A48u;   // 0, 1, 2, 3 | 4, 5, 6, 7
+  constexpr uint32_t N0 = 0xCACCCED0u, N1 = 0xB8C0C4C8u;   // -8,-7,-6,-5 | -4,-3,-2,-1
+  const uint32_t idx = w & 0x7777u;
+  const uint32_t pos = prmt(P0, P1, idx);
+  const uint32_t neg = prmt(N0, N1, idx);
+  // 0xFF in byte i where nibble i is negative: selector 0xC (sign of byte 4 = 0x80) or 0x0
+  const uint32_t sg = w & 0x8888u;
+  const uint32_t mask = prmt(0u, 0x80u, sg | (sg >> 1));
+  return (neg & mask) | (pos & ~mask);
 }
 
-// The same 8 values as the E4M3 codes of q (one byte per element, in element order): the
-// 8-bit float operand form of the tensor cores' kind::f8f6f4, which holds every q in
-// [-8, 7] exactly.
-__device__ __forceinline__ uint2 quant_e4m3_8(const uint4& v, const QScale& qs) {
-  const __half2* h = reinterpret_cast<const __half2*>(&v);
-  uint32_t w[2];
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const float2 a = __half22float2(h[2 * i]), b = __half22float2(h[2 * i + 1]);
-    w[i] = e4m3_plus_zero(e4m3x2(quant1f(a.x, qs), quant1f(a.y, qs)) |
-                          (e4m3x2(quant1f(b.x, qs), quant1f(b.y, qs)) << 16));
-  }
-  return make_uint2(w[0], w[1]);
-}
-
-// Quantize 8 fp16 values against the group scale qs and pack them into 4 bytes (little-endian:
-// element 0 in the low nibble of byte 0).
-__device__ __forceinline__ uint32_t quant_pack8(const uint4& v, const QScale& qs) {
+// The exact rule (quant1) for 8 values, packed as below.
+__device__ __forceinline__ uint32_t quant_pack8_exact(const uint4& v, const QScale& qs) {
   const __half2* h = reinterpret_cast<const __half2*>(&v);
   uint32_t out = 0;
 #pragma unroll
@@ -109,10 +103,57 @@ __device__ __forceinline__ uint32_t quant_pack8(const uint4& v, const QScale& qs
   return out;
 }
 
+// Quantize 8 fp16 values against the group scale qs and pack them into 4 bytes (little-endian:
+// element 0 in the low nibble of byte 0).
+// Fast path, on the fp32 pipe alone: t = fl(f * r) differs from the exact quotient f / s by
+// at most 2^-19 (|f / s| <= 10.5 for every value of a group against its own scale), so
+// unless t lies within 2^-18 of a half-integer both round to the same integer.  t, clamped
+// to [-8, 7] (clamping and rounding commute), plus 1.5 * 2^23 is that integer rounded to
+// nearest even, held in two's complement in the low bits of the sum.  Near a half-integer
+// the exact rule decides (rare: a few values in a million of those a quantizer meets; a CPU
+// test checks the whole claim on every reachable (f, s) pair).  A zero scale has r = 0, so
+// every t is 0; a NaN t clamps to -8, as the exact rule's clamp gives.
+// FAST = false: the exact rule alone (a shorter dependency chain, for latency-bound callers).
+template <bool FAST = true>
+__device__ __forceinline__ uint32_t quant_pack8(const uint4& v, const QScale& qs) {
+  if constexpr (!FAST) return quant_pack8_exact(v, qs);
+  constexpr float kMagic = 12582912.0f;          // 1.5 * 2^23
+  constexpr float kNear = 0.5f - 0x1p-18f;
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
+  uint32_t y[8];
+  bool near = false;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(h[i]);
+    const float t0 = fminf(fmaxf(__fmul_rn(f.x, qs.r), -8.0f), 7.0f);
+    const float t1 = fminf(fmaxf(__fmul_rn(f.y, qs.r), -8.0f), 7.0f);
+    const float y0 = __fadd_rn(t0, kMagic), y1 = __fadd_rn(t1, kMagic);
+    near |= fabsf(__fsub_rn(t0, __fsub_rn(y0, kMagic))) >= kNear;
+    near |= fabsf(__fsub_rn(t1, __fsub_rn(y1, kMagic))) >= kNear;
+    y[2 * i] = __float_as_uint(y0);
+    y[2 * i + 1] = __float_as_uint(y1);
+  }
+  if (near) return quant_pack8_exact(v, qs);
+  // low bytes: q0 q2 q4 q6 and q1 q3 q5 q7
+  const uint32_t ev = prmt(prmt(y[0], y[2], 0x0040u), prmt(y[4], y[6], 0x0040u), 0x5410u);
+  const uint32_t od = prmt(prmt(y[1], y[3], 0x0040u), prmt(y[5], y[7], 0x0040u), 0x5410u);
+  return (ev & 0x0F0F0F0Fu) | ((od & 0x0F0F0F0Fu) << 4);
+}
+
+// The same 8 values as the E4M3 codes of q (one byte per element, in element order): the
+// 8-bit float operand form of the tensor cores' kind::f8f6f4, which holds every q in
+// [-8, 7] exactly.
+template <bool FAST = true>
+__device__ __forceinline__ uint2 quant_e4m3_8(const uint4& v, const QScale& qs) {
+  const uint32_t w = quant_pack8<FAST>(v, qs);
+  return make_uint2(e4m3_of_nibbles(w), e4m3_of_nibbles(w >> 16));
+}
+
 // The same 8 values as 16*q in signed bytes, in the GEMM's operand order: bytes 0..3 hold
 // elements 0,2,4,6 and bytes 4..7 elements 1,3,5,7 (what the GEMM makes of a packed word).
+template <bool FAST = true>
 __device__ __forceinline__ uint2 quant_expand8(const uint4& v, const QScale& qs) {
-  const uint32_t w = quant_pack8(v, qs);
+  const uint32_t w = quant_pack8<FAST>(v, qs);
   return make_uint2((w << 4) & 0xF0F0F0F0u, w & 0xF0F0F0F0u);
 }
 
@@ -121,15 +162,15 @@ __device__ __forceinline__ uint2 quant_expand8(const uint4& v, const QScale& qs)
 // bytes, element order, see quant_e4m3_8).
 enum QForm : int { FORM_PACKED = 0, FORM_EXPANDED = 1, FORM_E4M3 = 2 };
 
-template <int FORM>
+template <int FORM, bool FAST = true>
 __device__ __forceinline__ void store_quantized(uint32_t* dst, uint2* xdst, const uint4& v,
                                                 const QScale& qs) {
   if constexpr (FORM == FORM_EXPANDED)
-    *xdst = quant_expand8(v, qs);
+    *xdst = quant_expand8<FAST>(v, qs);
   else if constexpr (FORM == FORM_E4M3)
-    *xdst = quant_e4m3_8(v, qs);
+    *xdst = quant_e4m3_8<FAST>(v, qs);
   else
-    *dst = quant_pack8(v, qs);
+    *dst = quant_pack8<FAST>(v, qs);
 }
 
 // CH > 0: the group is exactly CH 128-wide chunks, kept in registers (one pass over HBM).
@@ -137,10 +178,12 @@ __device__ __forceinline__ void store_quantized(uint32_t* dst, uint2* xdst, cons
 // FORM: the output form (QForm).
 // Each half-warp takes UPT (row, group) units per round, all their loads issued before any
 // arithmetic, so that several 16-byte loads per thread are in flight (the kernel is bound by
-// memory latency, not by its arithmetic).  Units are indexed in 32 bits (the host launches
+// memory latency, not by its arithmetic).  FAST: the fast per-value path (quant_pack8), for
+// throughput; without it the exact rule alone, whose shorter chain suits a batch of a few
+// tokens, where each thread quantizes one group and the latency of that chain is the time.  Units are indexed in 32 bits (the host launches
 // this kernel only when rows * K / group < 2^31) and split into (row, group) by a shift when
 // the groups per row are a power of two (g_shift >= 0).
-template <int CH, int FORM = FORM_PACKED, int UPT = 1>
+template <int CH, int FORM = FORM_PACKED, int UPT = 1, bool FAST = true>
 __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __restrict__ x,
                                                             int64_t rows, int64_t K, int group,
                                                             uint8_t* __restrict__ packed,
@@ -202,7 +245,7 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __rest
                                                  (int64_t)g[u] * group) + lane16;
 #pragma unroll
           for (int c = 0; c < CH; ++c)
-            store_quantized<FORM>(dst + c * 16, xdst + c * 16, v[u][c], qs);
+            store_quantized<FORM, FAST>(dst + c * 16, xdst + c * 16, v[u][c], qs);
           if (lane16 == 0) scales[(int64_t)row[u] * G + g[u]] = s;
         }
       }
@@ -229,7 +272,7 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __rest
         uint2* xdst =
             reinterpret_cast<uint2*>(packed + (int64_t)row * K + (int64_t)g * group) + lane16;
         for (int c = 0; c < chunks; ++c)
-          store_quantized<FORM>(dst + c * 16, xdst + c * 16, __ldg(src + c * 16), qs);
+          store_quantized<FORM, FAST>(dst + c * 16, xdst + c * 16, __ldg(src + c * 16), qs);
         if (lane16 == 0) scales[(int64_t)row * G + g] = s;
       }
     }

@@ -97,7 +97,8 @@ apex_status_t apex_w4a4_gemm_expanded(int64_t M, int64_t N, int64_t K, int32_t g
  *   Its size should be apex_w4a4_gemm_workspace_size(...); a smaller one limits the
  *   split.  Its first bytes hold per-tile arrival counters that must be zero before the
  *   first use (e.g. cudaMemset); every call that completes leaves them zero again.  Calls
- *   that share a workspace must not run concurrently.
+ *   that share a workspace must not run concurrently, and a workspace used for one shape
+ *   (M, N, K, group sizes) must be zeroed again before it serves another.
  */
 apex_status_t apex_w4a4_gemm(int64_t M, int64_t N, int64_t K, int32_t group_a, int32_t group_w,
                              const void *a_packed, const void *a_scales, const void *w_packed,
