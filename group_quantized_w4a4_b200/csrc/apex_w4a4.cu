@@ -960,22 +960,32 @@ apex_status_t apex_quantize_act_int4_dual(const void* x_f16, int64_t M, int64_t 
       !aligned(x_scales_f16, 2) || !aligned(x_out_f16, 16))
     return APEX_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const unsigned nb = grid_for(((M * (K / 128) + 1) / 2) * 32, 128, 32);
+  const int64_t G = K / 128;
+  if (M * G >= (1ll << 31) || C >= 65536) return APEX_ERR_UNSUPPORTED;   // 32-bit units, 16-bit table
+  const int g_shift = (G & (G - 1)) == 0 ? __builtin_ctzll((unsigned long long)G) : -1;
+  const size_t tab = apex::dual_table_bytes(K);
+  if (tab > 200 * 1024) return APEX_ERR_UNSUPPORTED;
+  const unsigned nb = grid_for(((M * G + 1) / 2) * 32, 128, 32);
   const __half* xh = static_cast<const __half*>(x_f16);
   const int32_t* ch = static_cast<const int32_t*>(channels);
   uint8_t* q = static_cast<uint8_t*>(x_q);
   __half* sc = static_cast<__half*>(x_scales_f16);
   __half* xo = static_cast<__half*>(x_out_f16);
+  auto run = [&](auto kern) -> cudaError_t {
+    if (tab > 48 * 1024) {
+      const cudaError_t ea =
+          cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tab);
+      if (ea != cudaSuccess) return ea;
+    }
+    return launch_pdl(kern, nb, 128, tab, s, xh, M, K, ch, (int)C, q, sc, xo, (int)Cp, g_shift);
+  };
   cudaError_t e;
   if (form == APEX_FORM_FP8)
-    e = launch_pdl(apex::quantize_dual_kernel<apex::FORM_E4M3>, nb, 128, 0, s, xh, M, K, ch,
-                   (int)C, q, sc, xo, (int)Cp);
+    e = run(apex::quantize_dual_kernel<apex::FORM_E4M3>);
   else if (form == APEX_FORM_EXPANDED)
-    e = launch_pdl(apex::quantize_dual_kernel<apex::FORM_EXPANDED>, nb, 128, 0, s, xh, M, K, ch,
-                   (int)C, q, sc, xo, (int)Cp);
+    e = run(apex::quantize_dual_kernel<apex::FORM_EXPANDED>);
   else
-    e = launch_pdl(apex::quantize_dual_kernel<apex::FORM_PACKED>, nb, 128, 0, s, xh, M, K, ch,
-                   (int)C, q, sc, xo, (int)Cp);
+    e = run(apex::quantize_dual_kernel<apex::FORM_PACKED>);
   if (e != cudaSuccess) return APEX_ERR_CUDA;
   return cuda_status(cudaPeekAtLastError());
 }

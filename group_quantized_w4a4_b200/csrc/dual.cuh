@@ -12,8 +12,8 @@
 // The 16-bit product x_out . w_out^T runs inside the E4M3-carrier GEMM as extra K-steps of
 // each tile (gemm_f8.cuh), added to the fp32 accumulators before the single fp16 rounding.
 // The channel list is sorted ascending, distinct, each in [0, K) (the caller's contract;
-// entries outside a lane's range are skipped, so a bad list gives wrong values, never an
-// out-of-bounds access).
+// entries outside [0, K) are skipped and indices past the list are never written, so a bad
+// list gives wrong values, never an out-of-bounds access).
 #pragma once
 #include <cuda_fp16.h>
 #include <stdint.h>
@@ -22,17 +22,6 @@
 #include "quantize.cuh"
 
 namespace apex {
-
-// First index i in [0, C) with ch[i] >= k (C when there is none).
-__device__ __forceinline__ int lower_bound_ch(const int32_t* __restrict__ ch, int C, int k) {
-  int lo = 0, hi = C;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(ch + mid) < k) lo = mid + 1;
-    else hi = mid;
-  }
-  return lo;
-}
 
 // The fp16 bit pattern of element j (0..7) of 8 packed halves.
 __device__ __forceinline__ uint16_t half_bits_of(const uint4& v, int j) {
@@ -52,44 +41,64 @@ __device__ __forceinline__ void clear_halves(uint4& v, uint32_t m8) {
   v.w &= keep(3);
 }
 
+// Shared-memory bytes of quantize_dual_kernel's outlier table for K channels.
+__host__ __device__ constexpr size_t dual_table_bytes(int64_t K) { return (size_t)(K / 8) * 3; }
+
 // One half-warp per (row, 128-wide group), as quantize_pack_kernel<1, FORM>; each lane owns 8
-// consecutive channels.  Outlier channels of the lane are found in the sorted list (binary
-// search for the lane's first channel, then a short scan).
+// consecutive channels (a chunk).  Each block first turns the sorted channel list into a
+// table in shared memory: per chunk, a byte with the chunk's outlier channels set, and the
+// list index of its first outlier; a lane then finds its outliers with one lookup.  Units
+// are indexed in 32 bits (the host launches this kernel only when rows * K / 128 < 2^31),
+// split into (row, group) by a shift when K / 128 is a power of two (g_shift >= 0).
 template <int FORM>
 __global__ void __launch_bounds__(128) quantize_dual_kernel(
     const __half* __restrict__ x, int64_t rows, int64_t K, const int32_t* __restrict__ ch,
     int C, uint8_t* __restrict__ out, __half* __restrict__ scales,
-    __half* __restrict__ x_out, int Cp) {
+    __half* __restrict__ x_out, int Cp, int g_shift) {
+  extern __shared__ uint32_t s_tab[];
+  const uint32_t nchunk = (uint32_t)(K / 8);
+  uint32_t* s_mask = s_tab;                                           // [nchunk / 4]
+  uint16_t* s_first = reinterpret_cast<uint16_t*>(s_tab + nchunk / 4);  // [nchunk]
   grid_dep_wait();
   grid_dep_launch();
-  const int64_t G = K / 128;
-  const int64_t units = rows * G;
+  for (uint32_t w = threadIdx.x; w < nchunk / 4; w += blockDim.x) s_mask[w] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < C; i += blockDim.x) {
+    const int k = __ldg(ch + i);
+    if (k < 0 || k >= K) continue;
+    const uint32_t c = (uint32_t)k >> 3;
+    atomicOr(&s_mask[c >> 2], 1u << (8 * (c & 3) + (k & 7)));
+    if (i == 0 || (uint32_t)(__ldg(ch + i - 1) >> 3) != c) s_first[c] = (uint16_t)i;
+  }
+  __syncthreads();
+
+  const uint32_t G = (uint32_t)(K / 128);
+  const uint32_t units = (uint32_t)(rows * G);
   const int lane16 = threadIdx.x & 15;
-  const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t warps_total = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const uint32_t warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t warps_total = (gridDim.x * blockDim.x) >> 5;
   const int half = (threadIdx.x >> 4) & 1;
   uint16_t* xo = reinterpret_cast<uint16_t*>(x_out);
 
-  for (int64_t base = warp_global * 2; base < units; base += warps_total * 2) {
-    const int64_t unit = base + half;
+  for (uint32_t base = warp_global * 2; base < units; base += warps_total * 2) {
+    const uint32_t unit = base + half;
     const bool live = unit < units;
-    const int64_t row = live ? unit / G : 0;
-    const int64_t g = live ? unit % G : 0;
-    const int k0 = (int)(g * 128) + lane16 * 8;
-    uint4 v = live ? __ldg(reinterpret_cast<const uint4*>(x + row * K + k0))
+    const uint32_t u = live ? unit : 0u;
+    const uint32_t row = g_shift >= 0 ? u >> g_shift : u / G;
+    const uint32_t g = g_shift >= 0 ? u & (G - 1) : u - row * G;
+    const uint32_t c = g * 16 + lane16;                      // this lane's chunk
+    uint4 v = live ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)row * K) + c)
                    : make_uint4(0, 0, 0, 0);
     if (live) {
-      uint32_t m8 = 0;
-      for (int i = lower_bound_ch(ch, C, k0); i < C; ++i) {
-        const int k = __ldg(ch + i);
-        if (k >= k0 + 8) break;
-        if (k < k0) continue;
-        xo[row * Cp + i] = half_bits_of(v, k - k0);
-        m8 |= 1u << (k - k0);
+      const uint32_t m8 = (s_mask[c >> 2] >> (8 * (c & 3))) & 0xFFu;
+      if (m8) {
+        uint32_t i = s_first[c];
+        for (uint32_t b = m8; b; b &= b - 1, ++i)
+          if (i < (uint32_t)C) xo[(size_t)row * Cp + i] = half_bits_of(v, __ffs(b) - 1);
+        clear_halves(v, m8);
       }
-      clear_halves(v, m8);
       if (g == 0)   // the row's padding columns, once per row
-        for (int i = C + lane16; i < Cp; i += 16) xo[row * Cp + i] = 0;
+        for (int i = C + lane16; i < Cp; i += 16) xo[(size_t)row * Cp + i] = 0;
     }
     float amax = absmax8(v);
 #pragma unroll
@@ -98,9 +107,10 @@ __global__ void __launch_bounds__(128) quantize_dual_kernel(
     const __half s = group_scale(amax);
     const QScale qs = make_qscale(__half2float(s));
     if (live) {
-      store_quantized<FORM>(reinterpret_cast<uint32_t*>(out + row * (K / 2) + g * 64) + lane16,
-                            reinterpret_cast<uint2*>(out + row * K + g * 128) + lane16, v, qs);
-      if (lane16 == 0) scales[row * G + g] = s;
+      store_quantized<FORM>(
+          reinterpret_cast<uint32_t*>(out + (size_t)row * (K / 2) + (size_t)g * 64) + lane16,
+          reinterpret_cast<uint2*>(out + (size_t)row * K + (size_t)g * 128) + lane16, v, qs);
+      if (lane16 == 0) scales[(size_t)row * G + g] = s;
     }
   }
 }
