@@ -135,7 +135,9 @@ struct GemmCfg {
   static constexpr int KPS = stage_groups(BT);                     // K-groups per packed stage
   static constexpr int NBOX = KPS / 2;                             // 128-byte boxes per stage
   // operand slots (per group): expanded weight tile (tensor or shared memory) + token tile
-  static constexpr int NX = BT >= 128 ? (AQ8 ? 6 : 4) : 8;
+  // (16-token tiles: three hand-off units, so the converters can fill one while the MMAs of
+  // the two before it are still running; 12 x 32 + 8 x 16 columns fill the tensor memory)
+  static constexpr int NX = BT >= 128 ? (AQ8 ? 6 : 4) : BT == 16 ? 12 : 8;
   static constexpr int NSLOT = BT >= 128 ? (AQ8 ? 2 : 3) : KPS == 4 ? 8 : 4;
   // Epilogue: 8 warps.  Wide tiles split the 128 columns in two halves; narrow tiles run
   // two teams of 4 warps that take alternate hand-off units (so one team's TMEM loads and
