@@ -1073,9 +1073,12 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE, QOUT>::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (clustered) {
-    // no CTA of the cluster exits while stores into its shared memory may be in flight
+    // No CTA of the cluster exits before its partners have issued their stores into its
+    // shared memory.  Their arrival is counted on the owner's mbarrier, which the owner
+    // waits for on every path, so this barrier orders execution only: a relaxed arrive
+    // (a releasing one waits for this CTA's own global stores, measured 0.6 us per launch).
     if (!cl_waited) cluster_wait();
-    cluster_arrive();
+    cluster_arrive_relaxed();
     cluster_wait();
   }
   if (threadIdx.x == 0) trace_stamp(args, 5, 1);

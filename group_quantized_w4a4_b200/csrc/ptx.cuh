@@ -124,6 +124,10 @@ __device__ __forceinline__ bool mbar_wait2(uint32_t a, uint32_t pa, uint32_t b, 
 __device__ __forceinline__ void cluster_arrive() {
   asm volatile("barrier.cluster.arrive.release;" ::: "memory");
 }
+// Arrive without release semantics: for a barrier that orders execution only.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
 }
