@@ -353,8 +353,8 @@ cudaError_t quantize_launch_t(int64_t units, cudaStream_t s, const __half* xh, i
   const int64_t cap = (int64_t)dev_info().sms * 32;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  return launch_pdl(apex::quantize_pack_kernel<CH, FORM, UPT, FAST>, (unsigned)blocks, threads, 0, s,
-                    xh, rows, K, group, pk, sc, g_shift);
+  return launch_pdl(apex::quantize_pack_kernel<CH, FORM, UPT, FAST>, (unsigned)blocks, threads,
+                    0, s, xh, rows, K, group, pk, sc, g_shift);
 }
 
 template <int FORM>

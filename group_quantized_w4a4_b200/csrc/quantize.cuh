@@ -110,8 +110,8 @@ __device__ __forceinline__ uint32_t quant_pack8_exact(const uint4& v, const QSca
 // unless t lies within 2^-18 of a half-integer both round to the same integer.  t, clamped
 // to [-8, 7] (clamping and rounding commute), plus 1.5 * 2^23 is that integer rounded to
 // nearest even, held in two's complement in the low bits of the sum.  Near a half-integer
-// the exact rule decides (rare: a few values in a million of those a quantizer meets; a CPU
-// test checks the whole claim on every reachable (f, s) pair).  A zero scale has r = 0, so
+// the exact rule decides (under 0.1 % of all reachable (f, s) pairs; a CPU test enumerates
+// them all and checks the whole claim).  A zero scale has r = 0, so
 // every t is 0; a NaN t clamps to -8, as the exact rule's clamp gives.
 // FAST = false: the exact rule alone (a shorter dependency chain, for latency-bound callers).
 template <bool FAST = true>
@@ -180,9 +180,10 @@ __device__ __forceinline__ void store_quantized(uint32_t* dst, uint2* xdst, cons
 // arithmetic, so that several 16-byte loads per thread are in flight (the kernel is bound by
 // memory latency, not by its arithmetic).  FAST: the fast per-value path (quant_pack8), for
 // throughput; without it the exact rule alone, whose shorter chain suits a batch of a few
-// tokens, where each thread quantizes one group and the latency of that chain is the time.  Units are indexed in 32 bits (the host launches
-// this kernel only when rows * K / group < 2^31) and split into (row, group) by a shift when
-// the groups per row are a power of two (g_shift >= 0).
+// tokens, where each thread quantizes one group and the latency of that chain is the time.
+// Units are indexed in 32 bits (the host launches this kernel only when rows * K / group <
+// 2^31) and split into (row, group) by a shift when the groups per row are a power of two
+// (g_shift >= 0).
 template <int CH, int FORM = FORM_PACKED, int UPT = 1, bool FAST = true>
 __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half* __restrict__ x,
                                                             int64_t rows, int64_t K, int group,
