@@ -52,6 +52,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "ptx.cuh"
 #include "quantize.cuh"
 
@@ -649,6 +651,10 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE, QOUT>::THREADS, 1)
     // cluster mode: every tile is split over exactly `cluster` CTAs, the owner at rank 0
     bool expected = false;   // an owner: the parts' byte count is armed on rcv_full
     bool received = false;   // an owner: its partners' parts are in its shared memory
+    // Pairs (2-CTA clusters, plain output): each CTA finishes half of the tile's tokens
+    const bool PAIRS = !QOUT && args.cluster == 2;
+    constexpr int HALF = C::CPT / 2;
+    bool sent = false;       // a pair: this CTA's other half went to its peer
 
     // Scales of the 8-group block starting at gb8 of segment sg (this thread's token / row).
     auto block_scales = [&](const Seg& sg, int gb8, uint4& sa, uint4& sw) {
@@ -665,6 +671,33 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE, QOUT>::THREADS, 1)
     };
 
     float2 acc[C::CPT / 2];
+    // the pair's exchange with compile-time column offsets (acc stays in registers): send the
+    // columns [O, O + HALF) of acc to the peer, or add the received half into [O, O + HALF)
+    auto pair_send = [&](auto o_c, uint32_t dst, uint32_t bar) {
+      constexpr int O = decltype(o_c)::value;
+#pragma unroll
+      for (int e = 0; e < HALF; e += 4)
+        st_async_v4(dst + 4u * e, acc[(O + e) / 2].x, acc[(O + e) / 2].y,
+                    acc[(O + e) / 2 + 1].x, acc[(O + e) / 2 + 1].y, bar);
+    };
+    auto pair_add_write = [&](auto o_c, int m0t, int nn, bool nvalid_) {
+      constexpr int O = decltype(o_c)::value;
+      const float4* src = reinterpret_cast<const float4*>(s_rcv + (size_t)row * HALF);
+#pragma unroll
+      for (int e = 0; e < HALF; e += 4) {
+        const float4 v = src[e / 4];
+        acc[(O + e) / 2].x += v.x;
+        acc[(O + e) / 2].y += v.y;
+        acc[(O + e) / 2 + 1].x += v.z;
+        acc[(O + e) / 2 + 1].y += v.w;
+      }
+#pragma unroll
+      for (int e = 0; e < HALF; ++e) {
+        const int m = m0t + h * C::CPT + O + e;
+        const float v = ((O + e) & 1) ? acc[(O + e) / 2].y : acc[(O + e) / 2].x;
+        if (m < M && nvalid_) args.y[(size_t)m * N + nn] = __float2half_rn(v);
+      }
+    };
     // Where the finished tile is written: from one call site after the hand-off (always with
     // the quantized output; for 128-token tiles also without it, measured 2-3 % faster), or
     // in place at each hand-off path (narrow tiles: measured faster)
@@ -922,7 +955,32 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE, QOUT>::THREADS, 1)
         const int cf = args.streamk ? sk_owner(args, sg.t * args.S) : (int)blockIdx.x;
         const int cl = args.streamk ? sk_owner(args, sg.t * args.S + args.S - 1) : (int)blockIdx.x;
         bool owner_done = false;   // this CTA holds the whole tile now: write it
-        if (clustered) {
+        if (clustered && PAIRS) {
+          // A pair finishes the tile half each: this CTA sends its sums of the other half's
+          // tokens to its peer, adds the peer's sums of its own half and writes that half.
+          // (Two addends: the result does not depend on which CTA adds.)
+          const int cl_rank = (int)(blockIdx.x & 1u);
+          if (et == 0)
+            mbar_arrive_expect_tx(smem_u32(rcv_full), (uint32_t)(HALF * C::BM * 4));
+          expected = true;
+          cluster_wait();   // the peer's barriers are initialised
+          cl_waited = true;
+          {
+            const uint32_t dst =
+                cluster_map(smem_u32(s_rcv + (size_t)row * HALF), (uint32_t)(cl_rank ^ 1));
+            const uint32_t bar = cluster_map(smem_u32(rcv_full), (uint32_t)(cl_rank ^ 1));
+            if (cl_rank == 0) pair_send(std::integral_constant<int, HALF>{}, dst, bar);
+            else pair_send(std::integral_constant<int, 0>{}, dst, bar);
+          }
+          sent = true;
+          ok = mbar_wait_cluster(smem_u32(rcv_full), 0u, lim, abort_flag);
+          received = ok;
+          if (et == 0) trace_stamp(args, 15, 4 * k + 2);
+          aborted = bar_red_or(FB, NF, !ok);
+          if (aborted) break;
+          if (cl_rank == 0) pair_add_write(std::integral_constant<int, 0>{}, m0, n, nvalid);
+          else pair_add_write(std::integral_constant<int, HALF>{}, m0, n, nvalid);
+        } else if (clustered) {
           // The parts meet in the owner's shared memory.  A partner sends its part after the
           // segment loop (below), on every path; the owner takes them here, adds them in
           // CTA order and writes the tile.
@@ -1044,7 +1102,26 @@ __global__ void __launch_bounds__(GemmCfg<BT, MODE, QOUT>::THREADS, 1)
       have = have_next;
       sg = nx;
     }
-    if (clustered && team == 0) {
+    if (clustered && PAIRS && team == 0) {
+      // a CTA that gave up before its segment's end still sends its half (whatever it holds),
+      // so its peer's wait ends, and still takes its peer's half, so that no store into this
+      // CTA's shared memory is in flight when it exits
+      const int cl_rank = (int)(blockIdx.x & 1u);
+      if (!sent) {
+        if (!cl_waited) cluster_wait();
+        cl_waited = true;
+        const uint32_t dst =
+            cluster_map(smem_u32(s_rcv + (size_t)row * HALF), (uint32_t)(cl_rank ^ 1));
+        const uint32_t bar = cluster_map(smem_u32(rcv_full), (uint32_t)(cl_rank ^ 1));
+        if (cl_rank == 0) pair_send(std::integral_constant<int, HALF>{}, dst, bar);
+        else pair_send(std::integral_constant<int, 0>{}, dst, bar);
+      }
+      if (!received) {
+        if (et == 0 && !expected)
+          mbar_arrive_expect_tx(smem_u32(rcv_full), (uint32_t)(HALF * C::BM * 4));
+        mbar_wait_cluster(smem_u32(rcv_full), 0u, 2 * lim, never);
+      }
+    } else if (clustered && team == 0) {
       const int cl_rank = (int)(blockIdx.x % (unsigned)args.cluster);
       if (cl_rank != 0) {
         // A partner's part (its one segment's sums; whatever it holds if the CTA gave up)
