@@ -254,8 +254,9 @@ def test_gemm_split_k_is_deterministic(apex):
 @pytest.mark.parametrize("M,ways", [(16, 2), (16, 3), (16, 4), (32, 2), (5, 4)])
 def test_gemm_split_over_a_cluster_matches_oracle(apex, M, ways):
     # N chosen so that every tile is split `ways` ways on this device (one CTA per SM):
-    # 16- and 32-token tiles split 2-4 ways run as thread-block clusters that add the parts
-    # in the owner's shared memory.  The last tile is ragged.
+    # 16- and 32-token tiles split 2-4 ways run as thread-block clusters; a pair exchanges
+    # halves of its sums and each CTA writes half of the tile's tokens, larger clusters add
+    # the parts in the owner's shared memory.  The last tile is ragged.
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     N = 128 * (sms // ways) - 50
     K = 128 * 4 * ways * 2             # two pipeline stages per CTA
